@@ -1,0 +1,202 @@
+/*
+ * kivi.h - C ABI of the KIVI packed KV cache and its fused decode attention
+ * (libkivi.so, built for sm_100a).
+ *
+ * Method sources (cited by page title and section):
+ *   [KIVI page]   "KIVI: A Tuning-Free Asymmetric 2bit Quantization for KV Cache"
+ *                 (inference-research papers/kivi summary page): keys are
+ *                 quantized per channel, values per token, asymmetric 2-bit.
+ *   [HF page]     "KV cache quantization squeezes 5GB down to fit longer LLM
+ *                 generations": the cache grows with every generated token;
+ *                 quantization rounds values; keys per channel, values per token.
+ *   [Llama-3 rec] record "kv-efficiency/kivi-2bit-llama3-8b-gqa-8k", fields
+ *                 "Model" (32 layers, 8 kv heads, 32 query heads, head_dim 128),
+ *                 "KV bytes basis" (grouped history plus a full-precision
+ *                 residual of the most recent R tokens; the grouped term covers
+ *                 S-R tokens), "Methodology" (group size 32, residual length 128
+ *                 for both KIVI-2 and KIVI-4) and "notes" (4-bit byte count).
+ *
+ * Quantizer (one group of 32 values x, b bits): zero point mn = min(x),
+ * scale = (max(x) - mn) / (2^b - 1) in IEEE fp32, code = round-half-even(
+ * (x - mn) / scale) clamped to [0, 2^b - 1] (all codes 0 when scale == 0).
+ * The stored metadata is {fp16(scale), fp16(mn)}, both round-to-nearest-even;
+ * dequantized value = scale_h * code + mn_h.  Keys: one group per channel over
+ * 32 consecutive tokens.  Values: one group per token over 32 consecutive
+ * channels.
+ *
+ * Cache state of one layer holding S tokens (uniform over the batch):
+ *   NG(S) = max(0, floor((S - R) / G)) quantized groups cover tokens
+ *   [0, NG*G); tokens [NG*G, S) stay bf16 in a ring of R + G slots, token t at
+ *   slot t mod (R + G).  Appending token S flushes the oldest G ring tokens into
+ *   group NG exactly when S + 1 - NG*G == R + G, so NG after the append is
+ *   NG(S + 1).  G = 32 and R = 128 here.
+ *
+ * Packed layout (all little-endian, 32-bit code words):
+ *   records  [L][B][Hkv][NGcap] group records, NGcap = NG(max_tokens),
+ *            record bytes = G*D*b/4 + 8*D (3072 at D=128 b=2, 5120 at b=4,
+ *            1536 at D=64 b=2).  One record, in order:
+ *     K codes  G rows (token i of the group) x D*b/32 words; the code of
+ *              channel d sits at bit (d mod (32/b))*b of word d/(32/b).
+ *     V codes  D rows (channel d) x G*b/32 words; the code of token i sits at
+ *              bit (i mod (32/b))*b of word i/(32/b).  Each code array is
+ *              stored with the axis its attention product sums over innermost
+ *              (channels for q.k, tokens for p.v).
+ *     K meta   D entries {fp16 scale, fp16 min} (scale at the lower address),
+ *              entry d = channel d.
+ *     V meta   G * (D/32) entries {fp16 scale, fp16 min}, entry i*(D/32) + j =
+ *              token i, channels [32j, 32j + 32).
+ *   resid_k, resid_v  bf16 [L][B][Hkv][R + G][D].
+ *
+ * Conventions for every call below:
+ *   - Ownership: the caller allocates and frees every device buffer; the
+ *     library never allocates device memory.  The handle owns host state only
+ *     (config, pointers, token count S per layer).
+ *   - Device pointers are plain CUDA device addresses, contiguous row-major,
+ *     16-byte aligned.  `stream` is a cudaStream_t passed as void* (NULL =
+ *     legacy default stream).
+ *   - Calls are asynchronous on `stream`: they validate on the host, launch and
+ *     return.  KIVI_ERR_CUDA reports a launch error; device faults surface at
+ *     the caller's next synchronisation.  No exception crosses the ABI and the
+ *     library never exits the process.
+ *   - Inputs must be finite with |x| <= 65504 (fp16 metadata range); this is a
+ *     documented precondition, not checked on the device.
+ *   - One handle must not be used from two host threads at once; calls that
+ *     share a handle's workspace must be ordered on one stream.
+ */
+#ifndef KIVI_H
+#define KIVI_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KIVI_OK = 0,
+  KIVI_ERR_INVALID_ARG = 1,      /* null pointer, negative size, bad layer index */
+  KIVI_ERR_UNSUPPORTED = 2,      /* config outside the supported set (below) */
+  KIVI_ERR_BUFFER_TOO_SMALL = 3, /* a kivi_buffers size is below kivi_required_bytes */
+  KIVI_ERR_CAPACITY = 4,         /* the call would exceed max_tokens */
+  KIVI_ERR_STATE = 5,            /* prefill on a non-empty layer, append/attend on an empty one */
+  KIVI_ERR_CUDA = 6,             /* a CUDA runtime call or launch failed */
+  KIVI_ERR_DEVICE = 7            /* a kernel reported a failure in the device status word */
+} kivi_status;
+
+/* Cache geometry.  Supported: bits in {2, 4}, group_size == 32,
+ * residual == 128, head_dim in {64, 128}, num_q_heads a multiple of
+ * num_kv_heads with at most 8 query heads per kv head, all counts >= 1,
+ * max_tokens >= 1.  Query head h reads kv head h / (num_q_heads / num_kv_heads)
+ * (consecutive grouping, the usual repeat-KV convention; [Llama-3 rec] "Model"
+ * gives 32 query heads over 8 kv heads). */
+typedef struct {
+  int32_t batch;
+  int32_t num_layers;
+  int32_t num_kv_heads;
+  int32_t num_q_heads;
+  int32_t head_dim;
+  int32_t bits;
+  int32_t group_size;
+  int32_t residual;
+  int32_t max_tokens;
+} kivi_config;
+
+typedef struct {
+  size_t records_bytes;   /* group records of all layers */
+  size_t resid_k_bytes;   /* bf16 key ring of all layers */
+  size_t resid_v_bytes;   /* bf16 value ring of all layers */
+  size_t workspace_bytes; /* split-K partials and the device status word */
+} kivi_sizes;
+
+typedef struct {
+  void* records;
+  void* resid_k;
+  void* resid_v;
+  void* workspace;
+  kivi_sizes sizes;       /* the sizes the caller actually allocated */
+} kivi_buffers;
+
+typedef struct kivi_cache kivi_cache; /* opaque host handle */
+
+/* Device bytes each buffer needs for `cfg`.  Host only.
+ * Errors: INVALID_ARG (null), UNSUPPORTED (config outside the supported set). */
+kivi_status kivi_required_bytes(const kivi_config* cfg, kivi_sizes* out);
+
+/* Creates a handle over caller-owned buffers; every layer starts empty (S = 0).
+ * Zeroes the device status word in `workspace` with a synchronous cudaMemset.
+ * Errors: INVALID_ARG, UNSUPPORTED, BUFFER_TOO_SMALL, CUDA. */
+kivi_status kivi_cache_create(const kivi_config* cfg, const kivi_buffers* bufs,
+                              kivi_cache** out);
+
+/* Frees the host handle (not the caller's device buffers).  NULL is a no-op. */
+void kivi_cache_destroy(kivi_cache* cache);
+
+/* Token count S and quantized-group count NG(S) of `layer`.  Host only. */
+kivi_status kivi_cache_length(const kivi_cache* cache, int32_t layer,
+                              int32_t* S, int32_t* NG);
+
+/* Marks `layer` empty again (S = 0).  Host only; device contents are left as
+ * they are and are overwritten by the next prefill. */
+kivi_status kivi_cache_reset(kivi_cache* cache, int32_t layer);
+
+/* Prefill of one layer with S prompt tokens ([HF page]: the history that is
+ * quantized; [Llama-3 rec] "KV bytes basis": grouped history plus residual).
+ * k, v: device bf16 [B][Hkv][S][D].  Quantizes NG(S) groups of keys (per
+ * channel) and values (per token) into records 0..NG-1 and copies tokens
+ * [NG*G, S) into the rings.  S may be 0..max_tokens.
+ * Errors: INVALID_ARG, STATE (layer not empty), CAPACITY (S > max_tokens), CUDA. */
+kivi_status kivi_quantize_prefill(kivi_cache* cache, int32_t layer,
+                                  const void* k, const void* v, int32_t S,
+                                  void* stream);
+
+/* Appends one generated token per sequence to `layer` ([HF page]: the cache
+ * grows with every generated token).  k_new, v_new: device bf16 [B][Hkv][D],
+ * written to ring slot S mod (R+G).  When S + 1 - NG*G == R + G the same launch
+ * quantizes ring tokens [NG*G, NG*G + G) into record NG (the residual flush).
+ * The layer need not have been prefilled (S may be 0).
+ * Errors: INVALID_ARG, CAPACITY (S + 1 > max_tokens), CUDA. */
+kivi_status kivi_append_token(kivi_cache* cache, int32_t layer,
+                              const void* k_new, const void* v_new, void* stream);
+
+/* Single-token decode attention of `layer` over all S cached tokens:
+ * quantized groups dequantized in registers and the bf16 residual, merged under
+ * one softmax ([KIVI page]: the per-channel/per-token split follows how the
+ * attention kernel reads memory).  q: device bf16 [B][Hq][D]; out: device fp32
+ * [B][Hq][D], out[b][h] = sum_t softmax_t(sm_scale * <q[b][h], k_t>) v_t over the
+ * dequantized keys/values of kv head h / (Hq/Hkv).  sm_scale <= 0 selects
+ * 1/sqrt(D).  Uses the handle's workspace (split-K partials).
+ * Errors: INVALID_ARG, STATE (S == 0), CUDA. */
+kivi_status kivi_decode_attention(const kivi_cache* cache, int32_t layer,
+                                  const void* q, float* out, float sm_scale,
+                                  void* stream);
+
+/* Synchronises `stream`, then reads and clears the device status word.
+ * Returns KIVI_ERR_DEVICE if a kernel recorded a failure (a bounded wait that
+ * ran out), KIVI_ERR_CUDA if the synchronisation failed, else KIVI_OK.
+ * `code_out` (may be NULL) receives the raw status word. */
+kivi_status kivi_check_device_status(kivi_cache* cache, void* stream,
+                                     uint32_t* code_out);
+
+/* KV-cache bytes per token of one sequence of `cfg` holding S >= 1 tokens, all
+ * layers, host only ([Llama-3 rec] "KV bytes basis" and "notes").
+ *   stored:     what this layout keeps: NG(S) group records (codes plus fp16
+ *               metadata) and r = S - NG(S)*G bf16 residual tokens, over S.
+ *   codes_only: the record's "exact stored amount": codes of the NG(S)*G grouped
+ *               tokens plus the r bf16 residual tokens, no metadata, over S
+ *               (18,176 B/token for the Llama-3-8B skeleton at 2 bits, S=8192).
+ *   convention: the record's convention: grouped codes counted over all S tokens
+ *               plus R residual tokens amortised over S (16,384 + 2,048 =
+ *               18,432 B/token for the same skeleton; 34,816 at 4 bits).
+ * Any output pointer may be NULL.  Errors: INVALID_ARG (S < 1), UNSUPPORTED. */
+kivi_status kivi_cache_bytes(const kivi_config* cfg, int32_t S, double* stored,
+                             double* codes_only, double* convention);
+
+/* Static text for a status code; never NULL. */
+const char* kivi_status_string(kivi_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KIVI_H */

@@ -1,0 +1,354 @@
+/*
+ * kivi_oracle.c - plain, slow, CPU reference of the KIVI cache and decode
+ * attention.  TEST INFRASTRUCTURE ONLY: the tests, the package's smoke check
+ * and the benchmark's CPU-baseline leg may call it; the library path never
+ * does.  It shares no code, header or table with the CUDA library: the packed
+ * layout below is written here again from its definition.
+ *
+ * Sources (page title and section):
+ *   [KIVI page]   "KIVI: A Tuning-Free Asymmetric 2bit Quantization for KV Cache":
+ *                 keys quantized per channel, values per token, asymmetric.
+ *   [HF page]     "KV cache quantization squeezes 5GB down to fit longer LLM
+ *                 generations": keys per channel, values per token; quantization
+ *                 rounds values.
+ *   [Llama-3 rec] "kv-efficiency/kivi-2bit-llama3-8b-gqa-8k", fields "Model",
+ *                 "KV bytes basis", "Methodology": group size 32, residual 128,
+ *                 the most recent R tokens kept in full precision, the grouped
+ *                 term covering S - R tokens.
+ *
+ * Readings where the pages are silent (each one is a choice, listed in the
+ * design notes): zero point = group min and scale = (max - min)/(2^b - 1) in
+ * IEEE fp32; codes round half to even and are clamped to [0, 2^b - 1]; a
+ * constant group has scale 0 and codes 0; metadata stored as fp16
+ * round-to-nearest-even; the residual slides (it always holds the newest
+ * r in [R, R + G) tokens once S >= R); softmax scale 1/sqrt(D) unless given.
+ *
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -shared -fPIC.
+ * Float expressions are evaluated in single precision (SSE, FLT_EVAL_METHOD 0).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------------ */
+/* Number formats                                                           */
+/* ------------------------------------------------------------------------ */
+
+/* bf16 -> fp32 is exact: the bf16 bits are the high half of the fp32 bits. */
+static float bf16_bits_to_float(uint16_t h) {
+  uint32_t u = (uint32_t)h << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return f;
+}
+
+/* Round half to even of a non-negative double r (exactly representable). */
+static double round_half_even_nonneg(double r) {
+  double f = floor(r);
+  double diff = r - f;
+  if (diff > 0.5) return f + 1.0;
+  if (diff < 0.5) return f;
+  return (fmod(f, 2.0) == 0.0) ? f : f + 1.0;
+}
+
+/* fp32 -> IEEE binary16 bits, round to nearest, ties to even.  Binary16 has an
+ * 11-bit significand for |v| >= 2^-14 and a fixed quantum of 2^-24 below it;
+ * values that round to 65520 or more overflow to infinity. */
+uint16_t oracle_f32_to_f16_bits(float x) {
+  uint16_t sign = signbit(x) ? 0x8000u : 0u;
+  double a = fabs((double)x);
+  if (isnan(x)) return (uint16_t)(sign | 0x7e00u);
+  if (isinf(x)) return (uint16_t)(sign | 0x7c00u);
+  if (a == 0.0) return sign;
+  int e2;
+  frexp(a, &e2);          /* a = m * 2^e2, m in [0.5, 1) -> floor(log2 a) = e2 - 1 */
+  int e = e2 - 1;
+  if (e < -14) e = -14;   /* subnormal range shares the quantum of the lowest binade */
+  double quantum = ldexp(1.0, e - 10);
+  double n = round_half_even_nonneg(a / quantum); /* a / quantum is exact */
+  double v = n * quantum;
+  if (v >= 65520.0) return (uint16_t)(sign | 0x7c00u);
+  if (v < ldexp(1.0, -14)) {
+    return (uint16_t)(sign | (uint16_t)(v / ldexp(1.0, -24)));
+  }
+  frexp(v, &e2);
+  int ev = e2 - 1;                                  /* v may have moved up a binade */
+  uint32_t mant = (uint32_t)(v / ldexp(1.0, ev - 10)) - 1024u;
+  return (uint16_t)(sign | (uint16_t)((ev + 15) << 10) | (uint16_t)mant);
+}
+
+/* IEEE binary16 bits -> double (exact). */
+double oracle_f16_bits_to_double(uint16_t h) {
+  int sign = (h >> 15) & 1;
+  int exp = (h >> 10) & 0x1f;
+  int mant = h & 0x3ff;
+  double v;
+  if (exp == 0) v = ldexp((double)mant, -24);
+  else if (exp == 31) v = mant ? NAN : INFINITY;
+  else v = ldexp((double)(1024 + mant), exp - 25);
+  return sign ? -v : v;
+}
+
+/* ------------------------------------------------------------------------ */
+/* The asymmetric quantizer ([KIVI page] title, [HF page]: "asymmetric")    */
+/* ------------------------------------------------------------------------ */
+
+/* Quantizes n values x[0], x[stride], ... with b bits.  Outputs the fp32 scale
+ * and zero point and one code per value. */
+void oracle_quantize_group(const float* x, int n, int stride, int bits,
+                           float* scale_out, float* mn_out, uint8_t* codes) {
+  float mn = x[0], mx = x[0];
+  for (int i = 1; i < n; ++i) {
+    float v = x[(size_t)i * stride];
+    if (v < mn) mn = v;
+    if (v > mx) mx = v;
+  }
+  const int qmax = (1 << bits) - 1;
+  float scale = (mx - mn) / (float)qmax;
+  for (int i = 0; i < n; ++i) {
+    int c = 0;
+    if (scale > 0.0f) {
+      float t = (x[(size_t)i * stride] - mn) / scale;
+      c = (int)round_half_even_nonneg((double)t); /* t >= 0, exact in double */
+      if (c > qmax) c = qmax;
+    }
+    codes[i] = (uint8_t)c;
+  }
+  *scale_out = scale;
+  *mn_out = mn;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Packed group record (layout definition of the library's header)          */
+/* ------------------------------------------------------------------------ */
+
+enum { ORACLE_G = 32, ORACLE_R = 128 };
+
+long oracle_record_bytes(int D, int bits) {
+  return (long)ORACLE_G * D * bits / 4 + 8L * D;
+}
+
+/* Number of quantized groups for S tokens: NG(S) = max(0, floor((S-R)/G))
+ * ([Llama-3 rec] "KV bytes basis": the grouped term covers S - R tokens). */
+int oracle_num_groups(int S) {
+  if (S < ORACLE_R) return 0;
+  return (S - ORACLE_R) / ORACLE_G;
+}
+
+static void put_code(uint32_t* words, int index, int bits, int code) {
+  int per_word = 32 / bits;
+  words[index / per_word] |= (uint32_t)code << ((index % per_word) * bits);
+}
+
+static void put_u16(uint8_t* p, uint16_t v) {
+  p[0] = (uint8_t)(v & 0xff);
+  p[1] = (uint8_t)(v >> 8);
+}
+
+/* Builds one group record from a key tile and a value tile of G tokens,
+ * each token a row of D bf16 values (row stride `ld` elements).
+ *   keys: one quantization group per channel over the G tokens ([KIVI page]
+ *         "KEYS ... PER-CHANNEL");
+ *   values: one group per token over each block of 32 channels ([KIVI page]
+ *         "VALUES ... PER-TOKEN"; group size 32 per [Llama-3 rec] "Methodology"). */
+void oracle_make_record(const uint16_t* k, const uint16_t* v, long ld, int D,
+                        int bits, uint8_t* record) {
+  const int G = ORACLE_G;
+  const long kc_words = (long)G * D * bits / 32;
+  memset(record, 0, (size_t)oracle_record_bytes(D, bits));
+  uint32_t* kcodes = (uint32_t*)malloc(sizeof(uint32_t) * kc_words);
+  uint32_t* vcodes = (uint32_t*)malloc(sizeof(uint32_t) * kc_words);
+  memset(kcodes, 0, sizeof(uint32_t) * kc_words);
+  memset(vcodes, 0, sizeof(uint32_t) * kc_words);
+  uint8_t* kmeta = record + 8L * kc_words;
+  uint8_t* vmeta = kmeta + 4L * D;
+
+  float col[ORACLE_G];
+  uint8_t codes[ORACLE_G];
+  /* Keys, per channel d over tokens 0..G-1. */
+  for (int d = 0; d < D; ++d) {
+    for (int i = 0; i < G; ++i) col[i] = bf16_bits_to_float(k[(long)i * ld + d]);
+    float scale, mn;
+    oracle_quantize_group(col, G, 1, bits, &scale, &mn, codes);
+    /* token-major rows of D*b/32 words: channel d of token i */
+    for (int i = 0; i < G; ++i) put_code(kcodes + (long)i * D * bits / 32, d, bits, codes[i]);
+    put_u16(kmeta + 4L * d, oracle_f32_to_f16_bits(scale));
+    put_u16(kmeta + 4L * d + 2, oracle_f32_to_f16_bits(mn));
+  }
+  /* Values, per token i over channel block j. */
+  float row[32];
+  for (int i = 0; i < G; ++i) {
+    for (int j = 0; j < D / 32; ++j) {
+      for (int c = 0; c < 32; ++c) row[c] = bf16_bits_to_float(v[(long)i * ld + 32 * j + c]);
+      float scale, mn;
+      oracle_quantize_group(row, 32, 1, bits, &scale, &mn, codes);
+      /* channel-major rows of G*b/32 words: token i of channel 32j+c */
+      for (int c = 0; c < 32; ++c)
+        put_code(vcodes + (long)(32 * j + c) * G * bits / 32, i, bits, codes[c]);
+      long e = (long)i * (D / 32) + j;
+      put_u16(vmeta + 4 * e, oracle_f32_to_f16_bits(scale));
+      put_u16(vmeta + 4 * e + 2, oracle_f32_to_f16_bits(mn));
+    }
+  }
+  for (long w = 0; w < kc_words; ++w) {
+    for (int byte = 0; byte < 4; ++byte) {
+      record[4 * w + byte] = (uint8_t)(kcodes[w] >> (8 * byte));
+      record[4 * kc_words + 4 * w + byte] = (uint8_t)(vcodes[w] >> (8 * byte));
+    }
+  }
+  free(kcodes);
+  free(vcodes);
+}
+
+/* Reads code `index` of a packed little-endian word row. */
+static int get_code(const uint8_t* row, int index, int bits) {
+  int per_word = 32 / bits;
+  const uint8_t* w = row + 4L * (index / per_word);
+  uint32_t word = (uint32_t)w[0] | ((uint32_t)w[1] << 8) | ((uint32_t)w[2] << 16) |
+                  ((uint32_t)w[3] << 24);
+  return (int)((word >> ((index % per_word) * bits)) & ((1u << bits) - 1u));
+}
+
+static uint16_t get_u16(const uint8_t* p) { return (uint16_t)(p[0] | (p[1] << 8)); }
+
+/* Dequantizes a record into key and value tiles [G][D] of doubles:
+ * x_hat = scale_h * code + min_h with the stored fp16 parameters. */
+void oracle_dequant_record(const uint8_t* record, int D, int bits, double* k_hat,
+                           double* v_hat) {
+  const int G = ORACLE_G;
+  const long row_words_k = (long)D * bits / 32;
+  const long row_words_v = (long)G * bits / 32;
+  const long kc_bytes = 4L * G * row_words_k;
+  const uint8_t* kmeta = record + 2 * kc_bytes;
+  const uint8_t* vmeta = kmeta + 4L * D;
+  for (int i = 0; i < G; ++i) {
+    for (int d = 0; d < D; ++d) {
+      int ck = get_code(record + 4L * row_words_k * i, d, bits);
+      double sk = oracle_f16_bits_to_double(get_u16(kmeta + 4L * d));
+      double mk = oracle_f16_bits_to_double(get_u16(kmeta + 4L * d + 2));
+      k_hat[(long)i * D + d] = sk * ck + mk;
+      int cv = get_code(record + kc_bytes + 4L * row_words_v * d, i, bits);
+      long e = (long)i * (D / 32) + d / 32;
+      double sv = oracle_f16_bits_to_double(get_u16(vmeta + 4 * e));
+      double mv = oracle_f16_bits_to_double(get_u16(vmeta + 4 * e + 2));
+      v_hat[(long)i * D + d] = sv * cv + mv;
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Cache state of one layer                                                 */
+/*   records [B][Hkv][NGcap][record bytes]; rings [B][Hkv][R+G][D] bf16      */
+/* ------------------------------------------------------------------------ */
+
+/* Prefill with S tokens: k, v are [B][Hkv][S][D] bf16. */
+void oracle_prefill(const uint16_t* k, const uint16_t* v, int B, int Hkv, int S, int D,
+                    int bits, int NGcap, uint8_t* records, uint16_t* ring_k,
+                    uint16_t* ring_v) {
+  const int G = ORACLE_G, slots = ORACLE_R + ORACLE_G;
+  const int NG = oracle_num_groups(S);
+  const long rb = oracle_record_bytes(D, bits);
+  for (int b = 0; b < B; ++b) {
+    for (int h = 0; h < Hkv; ++h) {
+      const long seq = (long)b * Hkv + h;
+      const uint16_t* kseq = k + seq * S * D;
+      const uint16_t* vseq = v + seq * S * D;
+      for (int g = 0; g < NG; ++g)
+        oracle_make_record(kseq + (long)g * G * D, vseq + (long)g * G * D, D, D, bits,
+                           records + (seq * NGcap + g) * rb);
+      for (int t = NG * G; t < S; ++t) {
+        memcpy(ring_k + (seq * slots + t % slots) * D, kseq + (long)t * D, 2L * D);
+        memcpy(ring_v + (seq * slots + t % slots) * D, vseq + (long)t * D, 2L * D);
+      }
+    }
+  }
+}
+
+/* Appends token S (k_new, v_new are [B][Hkv][D] bf16) to a layer holding S
+ * tokens; flushes the oldest G residual tokens into group NG(S) when the
+ * residual reaches R + G tokens.  Returns the new token count S + 1. */
+int oracle_append(const uint16_t* k_new, const uint16_t* v_new, int B, int Hkv, int S,
+                  int D, int bits, int NGcap, uint8_t* records, uint16_t* ring_k,
+                  uint16_t* ring_v) {
+  const int G = ORACLE_G, slots = ORACLE_R + ORACLE_G;
+  const int NG = oracle_num_groups(S);
+  const long rb = oracle_record_bytes(D, bits);
+  const int flush = (S + 1 - NG * G == slots);
+  for (int b = 0; b < B; ++b) {
+    for (int h = 0; h < Hkv; ++h) {
+      const long seq = (long)b * Hkv + h;
+      memcpy(ring_k + (seq * slots + S % slots) * D, k_new + seq * D, 2L * D);
+      memcpy(ring_v + (seq * slots + S % slots) * D, v_new + seq * D, 2L * D);
+      if (flush) {
+        const long first = (long)(NG * G) % slots; /* a whole group never wraps */
+        oracle_make_record(ring_k + (seq * slots + first) * D,
+                           ring_v + (seq * slots + first) * D, D, D, bits,
+                           records + (seq * NGcap + NG) * rb);
+      }
+    }
+  }
+  return S + 1;
+}
+
+/* Decode attention of one query head over one kv head holding S tokens:
+ * scores s_t = sm_scale * <q, k_hat_t>, out = sum_t softmax(s)_t v_hat_t, in
+ * double.  k_hat/v_hat are the dequantized groups for t < NG*G and the bf16
+ * residual otherwise. */
+void oracle_attend_one(const uint8_t* seq_records, const uint16_t* seq_ring_k,
+                       const uint16_t* seq_ring_v, const uint16_t* q, int S, int D,
+                       int bits, double sm_scale, double* out) {
+  const int G = ORACLE_G, slots = ORACLE_R + ORACLE_G;
+  const int NG = oracle_num_groups(S);
+  const long rb = oracle_record_bytes(D, bits);
+  double* K = (double*)malloc(sizeof(double) * (size_t)S * D);
+  double* V = (double*)malloc(sizeof(double) * (size_t)S * D);
+  double* s = (double*)malloc(sizeof(double) * (size_t)(S > 0 ? S : 1));
+  for (int g = 0; g < NG; ++g)
+    oracle_dequant_record(seq_records + g * rb, D, bits, K + (long)g * G * D,
+                          V + (long)g * G * D);
+  for (int t = NG * G; t < S; ++t) {
+    for (int d = 0; d < D; ++d) {
+      K[(long)t * D + d] = bf16_bits_to_float(seq_ring_k[(long)(t % slots) * D + d]);
+      V[(long)t * D + d] = bf16_bits_to_float(seq_ring_v[(long)(t % slots) * D + d]);
+    }
+  }
+  double m = -INFINITY;
+  for (int t = 0; t < S; ++t) {
+    double acc = 0.0;
+    for (int d = 0; d < D; ++d) acc += (double)bf16_bits_to_float(q[d]) * K[(long)t * D + d];
+    s[t] = sm_scale * acc;
+    if (s[t] > m) m = s[t];
+  }
+  double denom = 0.0;
+  for (int t = 0; t < S; ++t) {
+    s[t] = exp(s[t] - m);
+    denom += s[t];
+  }
+  for (int d = 0; d < D; ++d) {
+    double acc = 0.0;
+    for (int t = 0; t < S; ++t) acc += s[t] * V[(long)t * D + d];
+    out[d] = acc / denom;
+  }
+  free(K);
+  free(V);
+  free(s);
+}
+
+/* Decode attention of a whole layer: q [B][Hq][D] bf16 -> out [B][Hq][D]
+ * double.  Query head h reads kv head h / (Hq / Hkv). */
+void oracle_attention(const uint8_t* records, const uint16_t* ring_k,
+                      const uint16_t* ring_v, const uint16_t* q, int B, int Hkv, int Hq,
+                      int S, int D, int bits, int NGcap, double sm_scale, double* out) {
+  const int slots = ORACLE_R + ORACLE_G;
+  const long rb = oracle_record_bytes(D, bits);
+  const int per_kv = Hq / Hkv;
+  for (int b = 0; b < B; ++b) {
+    for (int h = 0; h < Hq; ++h) {
+      const long seq = (long)b * Hkv + h / per_kv;
+      oracle_attend_one(records + seq * NGcap * rb, ring_k + seq * slots * D,
+                        ring_v + seq * slots * D, q + ((long)b * Hq + h) * D, S, D, bits,
+                        sm_scale, out + ((long)b * Hq + h) * D);
+    }
+  }
+}

@@ -1,0 +1,201 @@
+"""KIVI packed KV cache with fused decode attention for B200 (sm_100a).
+
+A thin binding of the C ABI in ``include/kivi.h`` (``libkivi.so``): the
+functions below carry the C names and only marshal arguments; every step of the
+path runs in the library's CUDA kernels.  PyTorch supplies device memory and
+streams.  There is no CPU fallback: if the library is missing, calls raise.
+
+``KiviCache`` is a convenience owner of the device buffers (allocated with
+torch) around one handle.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from ._native import KiviBuffers, KiviConfig, KiviError, KiviSizes, check, lib
+
+__all__ = [
+    "KiviCache", "KiviConfig", "KiviError", "make_config",
+    "kivi_required_bytes", "kivi_cache_create", "kivi_cache_destroy", "kivi_cache_length",
+    "kivi_cache_reset", "kivi_quantize_prefill", "kivi_append_token", "kivi_decode_attention",
+    "kivi_check_device_status", "kivi_cache_bytes", "kivi_status_string",
+]
+
+GROUP_SIZE = 32
+RESIDUAL = 128
+
+
+def make_config(*, batch, num_layers, num_kv_heads, num_q_heads, head_dim, bits, max_tokens,
+                group_size=GROUP_SIZE, residual=RESIDUAL) -> KiviConfig:
+    return KiviConfig(batch, num_layers, num_kv_heads, num_q_heads, head_dim, bits,
+                      group_size, residual, max_tokens)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t: torch.Tensor | None, dtype=None, name="tensor") -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def kivi_required_bytes(cfg: KiviConfig) -> KiviSizes:
+    out = KiviSizes()
+    check(lib().kivi_required_bytes(ctypes.byref(cfg), ctypes.byref(out)), "kivi_required_bytes")
+    return out
+
+
+def kivi_cache_create(cfg: KiviConfig, buffers: KiviBuffers) -> int:
+    h = ctypes.c_void_p()
+    check(lib().kivi_cache_create(ctypes.byref(cfg), ctypes.byref(buffers), ctypes.byref(h)),
+          "kivi_cache_create")
+    return h.value
+
+
+def kivi_cache_destroy(handle: int) -> None:
+    lib().kivi_cache_destroy(handle)
+
+
+def kivi_cache_length(handle: int, layer: int) -> tuple[int, int]:
+    S, NG = ctypes.c_int32(), ctypes.c_int32()
+    check(lib().kivi_cache_length(handle, layer, ctypes.byref(S), ctypes.byref(NG)),
+          "kivi_cache_length")
+    return S.value, NG.value
+
+
+def kivi_cache_reset(handle: int, layer: int) -> None:
+    check(lib().kivi_cache_reset(handle, layer), "kivi_cache_reset")
+
+
+def kivi_quantize_prefill(handle: int, layer: int, k: torch.Tensor, v: torch.Tensor,
+                          S: int | None = None, stream=None) -> None:
+    """k, v: bf16 [B][Hkv][S][D] on the device."""
+    S = k.shape[2] if S is None else S
+    check(lib().kivi_quantize_prefill(handle, layer, _ptr(k, torch.bfloat16, "k"),
+                                      _ptr(v, torch.bfloat16, "v"), S, _stream(stream)),
+          "kivi_quantize_prefill")
+
+
+def kivi_append_token(handle: int, layer: int, k_new: torch.Tensor, v_new: torch.Tensor,
+                      stream=None) -> None:
+    """k_new, v_new: bf16 [B][Hkv][D] on the device."""
+    check(lib().kivi_append_token(handle, layer, _ptr(k_new, torch.bfloat16, "k_new"),
+                                  _ptr(v_new, torch.bfloat16, "v_new"), _stream(stream)),
+          "kivi_append_token")
+
+
+def kivi_decode_attention(handle: int, layer: int, q: torch.Tensor, out: torch.Tensor,
+                          sm_scale: float = 0.0, stream=None) -> torch.Tensor:
+    """q: bf16 [B][Hq][D]; out: fp32 [B][Hq][D] (written)."""
+    check(lib().kivi_decode_attention(handle, layer, _ptr(q, torch.bfloat16, "q"),
+                                      _ptr(out, torch.float32, "out"), float(sm_scale),
+                                      _stream(stream)),
+          "kivi_decode_attention")
+    return out
+
+
+def kivi_check_device_status(handle: int, stream=None) -> int:
+    code = ctypes.c_uint32()
+    rc = lib().kivi_check_device_status(handle, _stream(stream), ctypes.byref(code))
+    if rc not in (0, 7):
+        check(rc, "kivi_check_device_status")
+    return code.value
+
+
+def kivi_cache_bytes(cfg: KiviConfig, S: int) -> dict:
+    a, b, c = ctypes.c_double(), ctypes.c_double(), ctypes.c_double()
+    check(lib().kivi_cache_bytes(ctypes.byref(cfg), S, ctypes.byref(a), ctypes.byref(b),
+                                 ctypes.byref(c)), "kivi_cache_bytes")
+    return {"stored": a.value, "codes_only": b.value, "convention": c.value}
+
+
+def kivi_status_string(code: int) -> str:
+    return lib().kivi_status_string(code).decode()
+
+
+class KiviCache:
+    """Device buffers (torch allocations) plus one libkivi handle."""
+
+    def __init__(self, *, batch, num_layers, num_kv_heads, num_q_heads, head_dim, bits,
+                 max_tokens, device="cuda"):
+        self.cfg = make_config(batch=batch, num_layers=num_layers, num_kv_heads=num_kv_heads,
+                               num_q_heads=num_q_heads, head_dim=head_dim, bits=bits,
+                               max_tokens=max_tokens)
+        sizes = kivi_required_bytes(self.cfg)
+        dev = torch.device(device)
+        self.records = torch.empty(max(sizes.records_bytes, 16), dtype=torch.uint8, device=dev)
+        self.resid_k = torch.empty(sizes.resid_k_bytes, dtype=torch.uint8, device=dev)
+        self.resid_v = torch.empty(sizes.resid_v_bytes, dtype=torch.uint8, device=dev)
+        self.workspace = torch.empty(sizes.workspace_bytes, dtype=torch.uint8, device=dev)
+        bufs = KiviBuffers(self.records.data_ptr(), self.resid_k.data_ptr(),
+                           self.resid_v.data_ptr(), self.workspace.data_ptr(),
+                           KiviSizes(self.records.numel(), self.resid_k.numel(),
+                                     self.resid_v.numel(), self.workspace.numel()))
+        self.sizes = sizes
+        self.handle = kivi_cache_create(self.cfg, bufs)
+
+    # -- views of the packed state (for tests and inspection) --
+    def record_bytes(self) -> int:
+        return self.cfg.head_dim * (32 * self.cfg.bits // 4 + 8)
+
+    def ngcap(self) -> int:
+        return max(0, (self.cfg.max_tokens - RESIDUAL) // GROUP_SIZE)
+
+    def records_view(self, layer: int) -> torch.Tensor:
+        c = self.cfg
+        n = c.batch * c.num_kv_heads * self.ngcap() * self.record_bytes()
+        return self.records[layer * n:(layer + 1) * n].view(
+            c.batch, c.num_kv_heads, self.ngcap(), self.record_bytes())
+
+    def ring_view(self, which: str, layer: int) -> torch.Tensor:
+        c = self.cfg
+        buf = self.resid_k if which == "k" else self.resid_v
+        per_layer = c.batch * c.num_kv_heads * (RESIDUAL + GROUP_SIZE) * c.head_dim
+        return buf.view(torch.bfloat16)[layer * per_layer:(layer + 1) * per_layer].view(
+            c.batch, c.num_kv_heads, RESIDUAL + GROUP_SIZE, c.head_dim)
+
+    # -- calls --
+    def prefill(self, layer, k, v, stream=None):
+        kivi_quantize_prefill(self.handle, layer, k, v, stream=stream)
+
+    def append(self, layer, k_new, v_new, stream=None):
+        kivi_append_token(self.handle, layer, k_new, v_new, stream=stream)
+
+    def attend(self, layer, q, out=None, sm_scale=0.0, stream=None):
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        return kivi_decode_attention(self.handle, layer, q, out, sm_scale, stream=stream)
+
+    def length(self, layer):
+        return kivi_cache_length(self.handle, layer)
+
+    def reset(self, layer):
+        kivi_cache_reset(self.handle, layer)
+
+    def check_device_status(self, stream=None) -> int:
+        return kivi_check_device_status(self.handle, stream)
+
+    def close(self):
+        if getattr(self, "handle", None):
+            kivi_cache_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

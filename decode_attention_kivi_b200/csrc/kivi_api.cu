@@ -1,0 +1,284 @@
+// kivi_api.cu - the C ABI declared in include/kivi.h: validation, cache state
+// bookkeeping on the host, and kernel launches.  No device memory is allocated
+// here; the caller owns every buffer.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/kivi.h"
+#include "kivi_kernels.h"
+#include "kivi_layout.cuh"
+
+struct kivi_cache {
+  kivi_config cfg;
+  kivi_buffers bufs;
+  std::vector<int32_t> S;  // token count per layer
+  int ngcap;
+  long rec_bytes;
+  int max_splits;
+  int num_sms;
+  int device;
+};
+
+namespace {
+
+using kivi::kGroup;
+using kivi::kResidual;
+using kivi::kRingSlots;
+
+kivi_status validate_config(const kivi_config* c) {
+  if (!c) return KIVI_ERR_INVALID_ARG;
+  if (c->batch < 1 || c->num_layers < 1 || c->num_kv_heads < 1 || c->num_q_heads < 1 ||
+      c->max_tokens < 1 || c->head_dim < 1)
+    return KIVI_ERR_INVALID_ARG;
+  if (c->bits != 2 && c->bits != 4) return KIVI_ERR_UNSUPPORTED;
+  if (c->group_size != kGroup || c->residual != kResidual) return KIVI_ERR_UNSUPPORTED;
+  if (c->head_dim != 64 && c->head_dim != 128) return KIVI_ERR_UNSUPPORTED;
+  if (c->num_q_heads % c->num_kv_heads != 0) return KIVI_ERR_UNSUPPORTED;
+  const int hpk = c->num_q_heads / c->num_kv_heads;
+  if (hpk != 1 && hpk != 2 && hpk != 4 && hpk != 8) return KIVI_ERR_UNSUPPORTED;
+  return KIVI_OK;
+}
+
+long record_bytes(const kivi_config* c) {
+  return kivi::RecordGeom{c->head_dim, c->bits}.bytes();
+}
+
+kivi_sizes sizes_of(const kivi_config* c) {
+  kivi_sizes s;
+  const size_t seqs = (size_t)c->num_layers * c->batch * c->num_kv_heads;
+  const size_t ngcap = (size_t)kivi::num_groups(c->max_tokens);
+  s.records_bytes = seqs * ngcap * (size_t)record_bytes(c);
+  s.resid_k_bytes = seqs * kRingSlots * (size_t)c->head_dim * 2;
+  s.resid_v_bytes = s.resid_k_bytes;
+  const size_t parts = (size_t)c->batch * c->num_q_heads *
+                       kivi::max_splits(c->batch, c->num_kv_heads);
+  s.workspace_bytes = kivi::kWsHeader + parts * 2 * sizeof(float) +
+                      parts * (size_t)c->head_dim * sizeof(float);
+  return s;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+kivi_status check_layer(const kivi_cache* h, int32_t layer) {
+  if (!h) return KIVI_ERR_INVALID_ARG;
+  if (layer < 0 || layer >= h->cfg.num_layers) return KIVI_ERR_INVALID_ARG;
+  return KIVI_OK;
+}
+
+size_t layer_seqs(const kivi_cache* h) {
+  return (size_t)h->cfg.batch * h->cfg.num_kv_heads;
+}
+
+uint8_t* layer_records(const kivi_cache* h, int32_t layer) {
+  return static_cast<uint8_t*>(h->bufs.records) +
+         (size_t)layer * layer_seqs(h) * h->ngcap * h->rec_bytes;
+}
+
+__nv_bfloat16* layer_ring(const kivi_cache* h, void* base, int32_t layer) {
+  return static_cast<__nv_bfloat16*>(base) +
+         (size_t)layer * layer_seqs(h) * kRingSlots * h->cfg.head_dim;
+}
+
+kivi_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KIVI_OK : KIVI_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+kivi_status kivi_required_bytes(const kivi_config* cfg, kivi_sizes* out) {
+  if (!out) return KIVI_ERR_INVALID_ARG;
+  kivi_status st = validate_config(cfg);
+  if (st != KIVI_OK) return st;
+  *out = sizes_of(cfg);
+  return KIVI_OK;
+}
+
+kivi_status kivi_cache_create(const kivi_config* cfg, const kivi_buffers* bufs,
+                              kivi_cache** out) {
+  if (!out || !bufs) return KIVI_ERR_INVALID_ARG;
+  *out = nullptr;
+  kivi_status st = validate_config(cfg);
+  if (st != KIVI_OK) return st;
+  const kivi_sizes need = sizes_of(cfg);
+  if ((need.records_bytes && !bufs->records) || !bufs->resid_k || !bufs->resid_v ||
+      !bufs->workspace)
+    return KIVI_ERR_INVALID_ARG;
+  if ((bufs->records && !aligned16(bufs->records)) || !aligned16(bufs->resid_k) ||
+      !aligned16(bufs->resid_v) || !aligned16(bufs->workspace))
+    return KIVI_ERR_INVALID_ARG;
+  if (bufs->sizes.records_bytes < need.records_bytes ||
+      bufs->sizes.resid_k_bytes < need.resid_k_bytes ||
+      bufs->sizes.resid_v_bytes < need.resid_v_bytes ||
+      bufs->sizes.workspace_bytes < need.workspace_bytes)
+    return KIVI_ERR_BUFFER_TOO_SMALL;
+  int device = 0, sms = 0;
+  if (cudaGetDevice(&device) != cudaSuccess) return KIVI_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
+    return KIVI_ERR_CUDA;
+  if (cudaMemset(bufs->workspace, 0, kivi::kWsHeader) != cudaSuccess) return KIVI_ERR_CUDA;
+  kivi_cache* h = new (std::nothrow) kivi_cache();
+  if (!h) return KIVI_ERR_INVALID_ARG;
+  h->cfg = *cfg;
+  h->bufs = *bufs;
+  h->S.assign(cfg->num_layers, 0);
+  h->ngcap = kivi::num_groups(cfg->max_tokens);
+  h->rec_bytes = record_bytes(cfg);
+  h->max_splits = kivi::max_splits(cfg->batch, cfg->num_kv_heads);
+  h->num_sms = sms;
+  h->device = device;
+  *out = h;
+  return KIVI_OK;
+}
+
+void kivi_cache_destroy(kivi_cache* cache) { delete cache; }
+
+kivi_status kivi_cache_length(const kivi_cache* cache, int32_t layer, int32_t* S,
+                              int32_t* NG) {
+  kivi_status st = check_layer(cache, layer);
+  if (st != KIVI_OK) return st;
+  if (S) *S = cache->S[layer];
+  if (NG) *NG = kivi::num_groups(cache->S[layer]);
+  return KIVI_OK;
+}
+
+kivi_status kivi_cache_reset(kivi_cache* cache, int32_t layer) {
+  kivi_status st = check_layer(cache, layer);
+  if (st != KIVI_OK) return st;
+  cache->S[layer] = 0;
+  return KIVI_OK;
+}
+
+kivi_status kivi_quantize_prefill(kivi_cache* cache, int32_t layer, const void* k,
+                                  const void* v, int32_t S, void* stream) {
+  kivi_status st = check_layer(cache, layer);
+  if (st != KIVI_OK) return st;
+  if (S < 0) return KIVI_ERR_INVALID_ARG;
+  if (S > 0 && (!k || !v || !aligned16(k) || !aligned16(v))) return KIVI_ERR_INVALID_ARG;
+  if (cache->S[layer] != 0) return KIVI_ERR_STATE;
+  if (S > cache->cfg.max_tokens) return KIVI_ERR_CAPACITY;
+  if (S > 0) {
+    kivi::PrefillArgs a;
+    a.k = static_cast<const __nv_bfloat16*>(k);
+    a.v = static_cast<const __nv_bfloat16*>(v);
+    a.B = cache->cfg.batch;
+    a.Hkv = cache->cfg.num_kv_heads;
+    a.S = S;
+    a.ng = kivi::num_groups(S);
+    a.ngcap = cache->ngcap;
+    a.records = layer_records(cache, layer);
+    a.ring_k = layer_ring(cache, cache->bufs.resid_k, layer);
+    a.ring_v = layer_ring(cache, cache->bufs.resid_v, layer);
+    st = from_cuda(kivi::launch_prefill(cache->cfg.head_dim, cache->cfg.bits, a,
+                                        static_cast<cudaStream_t>(stream)));
+    if (st != KIVI_OK) return st;
+  }
+  cache->S[layer] = S;
+  return KIVI_OK;
+}
+
+kivi_status kivi_append_token(kivi_cache* cache, int32_t layer, const void* k_new,
+                              const void* v_new, void* stream) {
+  kivi_status st = check_layer(cache, layer);
+  if (st != KIVI_OK) return st;
+  if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return KIVI_ERR_INVALID_ARG;
+  const int S = cache->S[layer];
+  if (S + 1 > cache->cfg.max_tokens) return KIVI_ERR_CAPACITY;
+  const int ng = kivi::num_groups(S);
+  kivi::AppendArgs a;
+  a.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  a.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  a.B = cache->cfg.batch;
+  a.Hkv = cache->cfg.num_kv_heads;
+  a.S = S;
+  a.ngcap = cache->ngcap;
+  a.flush = (S + 1 - ng * kGroup == kRingSlots) ? 1 : 0;
+  a.ng = ng;
+  a.ring_k = layer_ring(cache, cache->bufs.resid_k, layer);
+  a.ring_v = layer_ring(cache, cache->bufs.resid_v, layer);
+  a.records = layer_records(cache, layer);
+  st = from_cuda(kivi::launch_append(cache->cfg.head_dim, cache->cfg.bits, a,
+                                     static_cast<cudaStream_t>(stream)));
+  if (st != KIVI_OK) return st;
+  cache->S[layer] = S + 1;
+  return KIVI_OK;
+}
+
+kivi_status kivi_decode_attention(const kivi_cache* cache, int32_t layer, const void* q,
+                                  float* out, float sm_scale, void* stream) {
+  kivi_status st = check_layer(cache, layer);
+  if (st != KIVI_OK) return st;
+  if (!q || !out || !aligned16(q) || !aligned16(out)) return KIVI_ERR_INVALID_ARG;
+  if (!std::isfinite(sm_scale)) return KIVI_ERR_INVALID_ARG;
+  if (cache->S[layer] == 0) return KIVI_ERR_STATE;
+  kivi::DecodeArgs a;
+  a.records = layer_records(cache, layer);
+  a.ring_k = layer_ring(cache, cache->bufs.resid_k, layer);
+  a.ring_v = layer_ring(cache, cache->bufs.resid_v, layer);
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.out = out;
+  uint8_t* ws = static_cast<uint8_t*>(cache->bufs.workspace);
+  const size_t parts = (size_t)cache->cfg.batch * cache->cfg.num_q_heads * cache->max_splits;
+  a.status = reinterpret_cast<uint32_t*>(ws);
+  a.ws_ml = reinterpret_cast<float*>(ws + kivi::kWsHeader);
+  a.ws_acc = a.ws_ml + 2 * parts;
+  a.B = cache->cfg.batch;
+  a.Hkv = cache->cfg.num_kv_heads;
+  a.Hq = cache->cfg.num_q_heads;
+  a.S = cache->S[layer];
+  a.ngcap = cache->ngcap;
+  a.sm_scale = sm_scale;
+  a.max_splits = cache->max_splits;
+  a.num_sms = cache->num_sms;
+  return from_cuda(kivi::launch_decode(cache->cfg.head_dim, cache->cfg.bits, a,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+kivi_status kivi_check_device_status(kivi_cache* cache, void* stream, uint32_t* code_out) {
+  if (!cache) return KIVI_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return KIVI_ERR_CUDA;
+  uint32_t code = 0;
+  if (cudaMemcpy(&code, cache->bufs.workspace, sizeof code, cudaMemcpyDeviceToHost) !=
+      cudaSuccess)
+    return KIVI_ERR_CUDA;
+  if (code != 0 && cudaMemset(cache->bufs.workspace, 0, sizeof code) != cudaSuccess)
+    return KIVI_ERR_CUDA;
+  if (code_out) *code_out = code;
+  return code ? KIVI_ERR_DEVICE : KIVI_OK;
+}
+
+kivi_status kivi_cache_bytes(const kivi_config* cfg, int32_t S, double* stored,
+                             double* codes_only, double* convention) {
+  kivi_status st = validate_config(cfg);
+  if (st != KIVI_OK) return st;
+  if (S < 1) return KIVI_ERR_INVALID_ARG;
+  const double lh = (double)cfg->num_layers * cfg->num_kv_heads;
+  const double codes_per_tok = lh * cfg->head_dim * 2.0 * cfg->bits / 8.0;
+  const double bf16_per_tok = lh * cfg->head_dim * 2.0 * 2.0;
+  const int ng = kivi::num_groups(S);
+  const int r = S - ng * kGroup;
+  if (stored) *stored = (ng * lh * (double)record_bytes(cfg) + r * bf16_per_tok) / S;
+  if (codes_only) *codes_only = ((double)ng * kGroup * codes_per_tok + r * bf16_per_tok) / S;
+  if (convention) *convention = codes_per_tok + kResidual * bf16_per_tok / S;
+  return KIVI_OK;
+}
+
+const char* kivi_status_string(kivi_status status) {
+  switch (status) {
+    case KIVI_OK: return "ok";
+    case KIVI_ERR_INVALID_ARG: return "invalid argument";
+    case KIVI_ERR_UNSUPPORTED: return "unsupported configuration";
+    case KIVI_ERR_BUFFER_TOO_SMALL: return "buffer smaller than kivi_required_bytes";
+    case KIVI_ERR_CAPACITY: return "cache capacity (max_tokens) exceeded";
+    case KIVI_ERR_STATE: return "call not valid in the layer's current state";
+    case KIVI_ERR_CUDA: return "CUDA runtime error";
+    case KIVI_ERR_DEVICE: return "a kernel reported a failure in the device status word";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

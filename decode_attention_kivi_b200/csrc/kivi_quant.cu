@@ -1,0 +1,228 @@
+// kivi_quant.cu - KIVI group quantization: prefill, residual copy, append with flush.
+//
+// The quantizer ("KIVI: A Tuning-Free Asymmetric 2bit Quantization for KV
+// Cache"; "asymmetric" also on "KV cache quantization squeezes 5GB down to fit
+// longer LLM generations"): zero point = group min, scale = (max - min) /
+// (2^b - 1) in IEEE fp32, code = round-half-even((x - min) / scale) clamped to
+// [0, 2^b - 1], all codes 0 when scale == 0; the record keeps {fp16 scale,
+// fp16 min} rounded to nearest even.  Keys: one group per channel over 32
+// tokens.  Values: one group per token over 32 channels.  Explicit _rn
+// intrinsics keep every step IEEE round-to-nearest so the codes are
+// reproducible bit for bit.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "kivi_kernels.h"
+#include "kivi_layout.cuh"
+
+namespace kivi {
+namespace {
+
+constexpr int kQuantThreads = 128;
+
+template <int D>
+struct QuantSmem {
+  __nv_bfloat16 k[kGroup][D];
+  __nv_bfloat16 v[kGroup][D];
+  uint8_t kc[kGroup][D];
+  uint8_t vc[kGroup][D];
+};
+
+__device__ __forceinline__ uint32_t pack_meta(float scale, float mn) {
+  const uint32_t s = __half_as_ushort(__float2half_rn(scale));
+  const uint32_t m = __half_as_ushort(__float2half_rn(mn));
+  return s | (m << 16);
+}
+
+// Codes of one group of values already reduced to (mn, scale).
+template <int BITS>
+__device__ __forceinline__ uint8_t quant_code(float x, float mn, float scale) {
+  constexpr int kQmax = (1 << BITS) - 1;
+  if (!(scale > 0.0f)) return 0;
+  int c = __float2int_rn(__fdiv_rn(__fsub_rn(x, mn), scale));
+  return (uint8_t)min(max(c, 0), kQmax);
+}
+
+// Loads 32 token rows of D bf16 (row stride `ld` elements) into a smem tile.
+template <int D>
+__device__ __forceinline__ void load_tile(__nv_bfloat16 (*dst)[D], const __nv_bfloat16* src,
+                                          long ld) {
+  constexpr int kVecPerRow = D * 2 / 16;
+  for (int i = threadIdx.x; i < kGroup * kVecPerRow; i += kQuantThreads) {
+    const int t = i / kVecPerRow, c = i % kVecPerRow;
+    reinterpret_cast<uint4*>(&dst[t][0])[c] =
+        reinterpret_cast<const uint4*>(src + (long)t * ld)[c];
+  }
+}
+
+// Quantizes the K and V tiles in smem into one group record at `rec`.
+template <int D, int BITS>
+__device__ void quantize_tiles_to_record(QuantSmem<D>& sm, uint32_t* __restrict__ rec) {
+  constexpr RecordGeom geo{D, BITS};
+  constexpr int kQmax = (1 << BITS) - 1;
+  constexpr int kCpw = geo.codes_per_word();
+  uint32_t* kmeta = rec + geo.k_meta_off() / 4;
+  uint32_t* vmeta = rec + geo.v_meta_off() / 4;
+  // Keys: per channel d over the 32 tokens.
+  for (int d = threadIdx.x; d < D; d += kQuantThreads) {
+    float mn = __bfloat162float(sm.k[0][d]), mx = mn;
+#pragma unroll 8
+    for (int t = 1; t < kGroup; ++t) {
+      const float x = __bfloat162float(sm.k[t][d]);
+      mn = x < mn ? x : mn;  // strict comparisons, first occurrence wins (signed zeros)
+      mx = x > mx ? x : mx;
+    }
+    const float scale = __fdiv_rn(__fsub_rn(mx, mn), (float)kQmax);
+#pragma unroll 8
+    for (int t = 0; t < kGroup; ++t) sm.kc[t][d] = quant_code<BITS>(__bfloat162float(sm.k[t][d]), mn, scale);
+    kmeta[d] = pack_meta(scale, mn);
+  }
+  // Values: per token t over channel block j.
+  constexpr int kBlocks = D / 32;
+  for (int p = threadIdx.x; p < kGroup * kBlocks; p += kQuantThreads) {
+    const int t = p / kBlocks, j = p % kBlocks;
+    float mn = __bfloat162float(sm.v[t][32 * j]), mx = mn;
+#pragma unroll 8
+    for (int c = 1; c < 32; ++c) {
+      const float x = __bfloat162float(sm.v[t][32 * j + c]);
+      mn = x < mn ? x : mn;
+      mx = x > mx ? x : mx;
+    }
+    const float scale = __fdiv_rn(__fsub_rn(mx, mn), (float)kQmax);
+#pragma unroll 8
+    for (int c = 0; c < 32; ++c)
+      sm.vc[t][32 * j + c] = quant_code<BITS>(__bfloat162float(sm.v[t][32 * j + c]), mn, scale);
+    vmeta[t * kBlocks + j] = pack_meta(scale, mn);
+  }
+  __syncthreads();
+  // Pack: K token-major rows (channels innermost), V channel-major rows (tokens innermost).
+  constexpr int kWords = geo.code_words();
+  for (int wi = threadIdx.x; wi < kWords; wi += kQuantThreads) {
+    const int t = wi / geo.k_row_words(), w = wi % geo.k_row_words();
+    uint32_t word = 0;
+#pragma unroll
+    for (int i = 0; i < kCpw; ++i) word |= (uint32_t)sm.kc[t][w * kCpw + i] << (i * BITS);
+    rec[wi] = word;
+  }
+  for (int wi = threadIdx.x; wi < kWords; wi += kQuantThreads) {
+    const int d = wi / geo.v_row_words(), w = wi % geo.v_row_words();
+    uint32_t word = 0;
+#pragma unroll
+    for (int i = 0; i < kCpw; ++i) word |= (uint32_t)sm.vc[w * kCpw + i][d] << (i * BITS);
+    rec[geo.v_codes_off() / 4 + wi] = word;
+  }
+}
+
+// Prefill: one CTA per (group, kv head, sequence).
+template <int D, int BITS>
+__global__ void __launch_bounds__(kQuantThreads)
+prefill_groups_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+                      int S, int Hkv, int ngcap, uint8_t* __restrict__ records) {
+  __shared__ __align__(16) QuantSmem<D> sm;
+  constexpr RecordGeom geo{D, BITS};
+  const int g = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const long seq = (long)b * Hkv + h;
+  const long src = (seq * S + (long)g * kGroup) * D;
+  load_tile<D>(sm.k, k + src, D);
+  load_tile<D>(sm.v, v + src, D);
+  __syncthreads();
+  uint8_t* rec = records + (seq * ngcap + g) * geo.bytes();
+  quantize_tiles_to_record<D, BITS>(sm, reinterpret_cast<uint32_t*>(rec));
+}
+
+// Copies prompt tokens [first, S) of every (sequence, kv head) into ring slots t mod (R+G).
+template <int D>
+__global__ void __launch_bounds__(kQuantThreads)
+copy_residual_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+                     int S, int first, int Hkv, __nv_bfloat16* __restrict__ ring_k,
+                     __nv_bfloat16* __restrict__ ring_v) {
+  constexpr int kVecPerRow = D * 2 / 16;
+  const int h = blockIdx.x, b = blockIdx.y;
+  const long seq = (long)b * Hkv + h;
+  const int n = S - first;
+  for (int i = threadIdx.x; i < n * kVecPerRow; i += kQuantThreads) {
+    const int t = first + i / kVecPerRow, c = i % kVecPerRow;
+    const long src = (seq * S + t) * D;
+    const long dst = (seq * kRingSlots + t % kRingSlots) * D;
+    reinterpret_cast<uint4*>(ring_k + dst)[c] = reinterpret_cast<const uint4*>(k + src)[c];
+    reinterpret_cast<uint4*>(ring_v + dst)[c] = reinterpret_cast<const uint4*>(v + src)[c];
+  }
+}
+
+// Append token S to every (sequence, kv head); with `flush`, quantize ring
+// tokens [first, first + 32) into record `ng`.
+template <int D, int BITS>
+__global__ void __launch_bounds__(kQuantThreads)
+append_kernel(const __nv_bfloat16* __restrict__ k_new, const __nv_bfloat16* __restrict__ v_new,
+              int S, int Hkv, int ngcap, int flush, int ng, __nv_bfloat16* __restrict__ ring_k,
+              __nv_bfloat16* __restrict__ ring_v, uint8_t* __restrict__ records) {
+  __shared__ __align__(16) QuantSmem<D> sm;
+  constexpr RecordGeom geo{D, BITS};
+  constexpr int kVecPerRow = D * 2 / 16;
+  const int h = blockIdx.x, b = blockIdx.y;
+  const long seq = (long)b * Hkv + h;
+  __nv_bfloat16* rk = ring_k + seq * kRingSlots * D;
+  __nv_bfloat16* rv = ring_v + seq * kRingSlots * D;
+  if (flush) {
+    const int first = (ng * kGroup) % kRingSlots;  // a group never wraps the ring
+    load_tile<D>(sm.k, rk + (long)first * D, D);
+    load_tile<D>(sm.v, rv + (long)first * D, D);
+  }
+  // The new token's slot is not one of the flushed group's 32 slots.
+  const int slot = S % kRingSlots;
+  for (int c = threadIdx.x; c < kVecPerRow; c += kQuantThreads) {
+    reinterpret_cast<uint4*>(rk + (long)slot * D)[c] =
+        reinterpret_cast<const uint4*>(k_new + seq * D)[c];
+    reinterpret_cast<uint4*>(rv + (long)slot * D)[c] =
+        reinterpret_cast<const uint4*>(v_new + seq * D)[c];
+  }
+  if (flush) {
+    __syncthreads();
+    uint8_t* rec = records + (seq * ngcap + ng) * geo.bytes();
+    quantize_tiles_to_record<D, BITS>(sm, reinterpret_cast<uint32_t*>(rec));
+  }
+}
+
+template <int D, int BITS>
+cudaError_t launch_prefill_t(const PrefillArgs& a, cudaStream_t stream) {
+  if (a.ng > 0) {
+    dim3 grid(a.ng, a.Hkv, a.B);
+    prefill_groups_kernel<D, BITS><<<grid, kQuantThreads, 0, stream>>>(a.k, a.v, a.S, a.Hkv,
+                                                                      a.ngcap, a.records);
+  }
+  if (a.S > a.ng * kGroup) {
+    dim3 grid(a.Hkv, a.B);
+    copy_residual_kernel<D><<<grid, kQuantThreads, 0, stream>>>(a.k, a.v, a.S, a.ng * kGroup,
+                                                               a.Hkv, a.ring_k, a.ring_v);
+  }
+  return cudaGetLastError();
+}
+
+template <int D, int BITS>
+cudaError_t launch_append_t(const AppendArgs& a, cudaStream_t stream) {
+  dim3 grid(a.Hkv, a.B);
+  append_kernel<D, BITS><<<grid, kQuantThreads, 0, stream>>>(a.k_new, a.v_new, a.S, a.Hkv,
+                                                            a.ngcap, a.flush, a.ng, a.ring_k,
+                                                            a.ring_v, a.records);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_prefill(int D, int bits, const PrefillArgs& a, cudaStream_t stream) {
+  if (D == 128 && bits == 2) return launch_prefill_t<128, 2>(a, stream);
+  if (D == 128 && bits == 4) return launch_prefill_t<128, 4>(a, stream);
+  if (D == 64 && bits == 2) return launch_prefill_t<64, 2>(a, stream);
+  if (D == 64 && bits == 4) return launch_prefill_t<64, 4>(a, stream);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_append(int D, int bits, const AppendArgs& a, cudaStream_t stream) {
+  if (D == 128 && bits == 2) return launch_append_t<128, 2>(a, stream);
+  if (D == 128 && bits == 4) return launch_append_t<128, 4>(a, stream);
+  if (D == 64 && bits == 2) return launch_append_t<64, 2>(a, stream);
+  if (D == 64 && bits == 4) return launch_append_t<64, 4>(a, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace kivi

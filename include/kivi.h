@@ -85,9 +85,8 @@ typedef enum {
 } kivi_status;
 
 /* Cache geometry.  Supported: bits in {2, 4}, group_size == 32,
- * residual == 128, head_dim in {64, 128}, num_q_heads a multiple of
- * num_kv_heads with at most 8 query heads per kv head, all counts >= 1,
- * max_tokens >= 1.  Query head h reads kv head h / (num_q_heads / num_kv_heads)
+ * residual == 128, head_dim in {64, 128}, num_q_heads / num_kv_heads in
+ * {1, 2, 4, 8} (exact multiple), all counts >= 1, max_tokens >= 1.  Query head h reads kv head h / (num_q_heads / num_kv_heads)
  * (consecutive grouping, the usual repeat-KV convention; [Llama-3 rec] "Model"
  * gives 32 query heads over 8 kv heads). */
 typedef struct {

@@ -1,0 +1,118 @@
+"""The C ABI on the host (CPU only): the library loads, exports every symbol the
+header declares, validates its arguments, and its host-side byte arithmetic
+agrees with the pages' numbers and with the oracle."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle as O
+from decode_attention_kivi_b200 import _native as N
+from decode_attention_kivi_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return N.lib()
+
+
+def _header_functions():
+    text = open(os.path.join(ROOT, "include", "kivi.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kivi_[a-z_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _header_functions()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def cfg(**kw):
+    base = dict(batch=16, num_layers=32, num_kv_heads=8, num_q_heads=32, head_dim=128, bits=2,
+                group_size=32, residual=128, max_tokens=8192 + 64)
+    base.update(kw)
+    return N.KiviConfig(*[base[f] for f, _ in N.KiviConfig._fields_])
+
+
+def test_required_bytes_layout(lib):
+    s = N.KiviSizes()
+    c = cfg()
+    assert lib.kivi_required_bytes(ctypes.byref(c), ctypes.byref(s)) == 0
+    ngcap = O.num_groups(c.max_tokens)
+    assert s.records_bytes == 32 * 16 * 8 * ngcap * 3072
+    assert s.resid_k_bytes == s.resid_v_bytes == 32 * 16 * 8 * 160 * 128 * 2
+    assert s.workspace_bytes >= 256 + 16 * 32 * (128 + 2) * 4
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("bits", 3, 2), ("group_size", 64, 2), ("residual", 64, 2), ("head_dim", 96, 2),
+    ("num_q_heads", 12, 2), ("num_q_heads", 24, 2), ("batch", 0, 1), ("max_tokens", 0, 1),
+])
+def test_rejects_bad_configs(lib, field, value, code):
+    s = N.KiviSizes()
+    c = cfg(**{field: value})
+    assert lib.kivi_required_bytes(ctypes.byref(c), ctypes.byref(s)) == code
+    assert lib.kivi_required_bytes(None, ctypes.byref(s)) == 1
+
+
+def test_create_validates_buffers_before_touching_the_device(lib):
+    c = cfg(num_layers=1, batch=1, max_tokens=1000)
+    s = N.KiviSizes()
+    assert lib.kivi_required_bytes(ctypes.byref(c), ctypes.byref(s)) == 0
+    fake = 1 << 20  # never dereferenced: the call fails on sizes first
+    small = N.KiviSizes(s.records_bytes - 1, s.resid_k_bytes, s.resid_v_bytes, s.workspace_bytes)
+    bufs = N.KiviBuffers(fake, fake, fake, fake, small)
+    h = ctypes.c_void_p()
+    assert lib.kivi_cache_create(ctypes.byref(c), ctypes.byref(bufs), ctypes.byref(h)) == 3
+    misaligned = N.KiviBuffers(fake + 4, fake, fake, fake, s)
+    assert lib.kivi_cache_create(ctypes.byref(c), ctypes.byref(misaligned), ctypes.byref(h)) == 1
+    nulls = N.KiviBuffers(None, None, None, None, s)
+    assert lib.kivi_cache_create(ctypes.byref(c), ctypes.byref(nulls), ctypes.byref(h)) == 1
+    assert not h.value
+
+
+def test_null_handle_calls_fail_cleanly(lib):
+    S = ctypes.c_int32()
+    assert lib.kivi_cache_length(None, 0, ctypes.byref(S), None) == 1
+    assert lib.kivi_cache_reset(None, 0) == 1
+    assert lib.kivi_quantize_prefill(None, 0, None, None, 0, None) == 1
+    assert lib.kivi_append_token(None, 0, None, None, None) == 1
+    assert lib.kivi_decode_attention(None, 0, None, None, 0.0, None) == 1
+    assert lib.kivi_check_device_status(None, None, None) == 1
+    lib.kivi_cache_destroy(None)
+
+
+def test_status_strings(lib):
+    for code in range(8):
+        assert lib.kivi_status_string(code)
+    assert lib.kivi_status_string(99) == b"unknown status"
+
+
+@pytest.mark.parametrize("bits,S", [(2, 8192), (4, 8192), (2, 4096), (2, 300), (4, 161)])
+def test_cache_bytes_agree_with_oracle(lib, bits, S):
+    c = cfg(bits=bits)
+    vals = [ctypes.c_double() for _ in range(3)]
+    assert lib.kivi_cache_bytes(ctypes.byref(c), S, *[ctypes.byref(v) for v in vals]) == 0
+    o = O.cache_bytes(32, 8, 128, bits, S)
+    assert vals[0].value == pytest.approx(o["stored"], rel=1e-15)
+    assert vals[1].value == pytest.approx(o["codes_only"], rel=1e-15)
+    assert vals[2].value == pytest.approx(o["convention"], rel=1e-15)
+
+
+def test_cache_bytes_pages_numbers(lib):
+    """The record's printed figures: 18,432 (convention) and 18,176 (exact) B/token at
+    2 bits, 34,816 at 4 bits, Llama-3-8B skeleton at 8,192 tokens."""
+    out = [ctypes.c_double() for _ in range(3)]
+    c = cfg(bits=2)
+    lib.kivi_cache_bytes(ctypes.byref(c), 8192, *[ctypes.byref(v) for v in out])
+    assert out[2].value == 18432 and out[1].value == 18176
+    c = cfg(bits=4)
+    lib.kivi_cache_bytes(ctypes.byref(c), 8192, None, None, ctypes.byref(out[2]))
+    assert out[2].value == 34816
+    assert lib.kivi_cache_bytes(ctypes.byref(c), 0, None, None, None) == 1

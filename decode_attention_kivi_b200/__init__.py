@@ -21,6 +21,7 @@ __all__ = [
     "kivi_required_bytes", "kivi_cache_create", "kivi_cache_destroy", "kivi_cache_length",
     "kivi_cache_reset", "kivi_quantize_prefill", "kivi_append_token", "kivi_decode_attention",
     "kivi_check_device_status", "kivi_cache_bytes", "kivi_status_string",
+    "kivi_decode_attention_static_scratch",
 ]
 
 GROUP_SIZE = 32
@@ -105,6 +106,25 @@ def kivi_decode_attention(handle: int, layer: int, q: torch.Tensor, out: torch.T
                                       _ptr(out, torch.float32, "out"), float(sm_scale),
                                       _stream(stream)),
           "kivi_decode_attention")
+    return out
+
+
+def kivi_decode_attention_static_scratch(cfg: KiviConfig, records: int, resid_k: int,
+                                         resid_v: int, layer: int, S: int, q: torch.Tensor,
+                                         out: torch.Tensor, sm_scale: float = 0.0,
+                                         stream=None) -> torch.Tensor:
+    """Decode attention for callers that cannot allocate device memory.
+
+    Takes the cache buffers (device addresses) and the layer's token count S
+    instead of a handle, and keeps its split-K partials in the library's static
+    device array (no workspace).  Calls whose kernels overlap on the GPU share
+    that array and race; serialise them.  The first call on a device sets the
+    array up and should come before any stream capture.
+    """
+    check(lib().kivi_decode_attention_static_scratch(
+        ctypes.byref(cfg), records, resid_k, resid_v, layer, S, _ptr(q, torch.bfloat16, "q"),
+        _ptr(out, torch.float32, "out"), float(sm_scale), _stream(stream)),
+        "kivi_decode_attention_static_scratch")
     return out
 
 

@@ -26,7 +26,9 @@ class KiviBuffers(ctypes.Structure):
 
 STATUS = {0: "KIVI_OK", 1: "KIVI_ERR_INVALID_ARG", 2: "KIVI_ERR_UNSUPPORTED",
           3: "KIVI_ERR_BUFFER_TOO_SMALL", 4: "KIVI_ERR_CAPACITY", 5: "KIVI_ERR_STATE",
-          6: "KIVI_ERR_CUDA", 7: "KIVI_ERR_DEVICE"}
+          6: "KIVI_ERR_CUDA", 7: "KIVI_ERR_DEVICE", 8: "KIVI_ERR_SCRATCH_LIMIT"}
+
+STATIC_SCRATCH_BYTES = 8 << 20  # KIVI_STATIC_SCRATCH_BYTES
 
 _lib = None
 
@@ -59,6 +61,8 @@ def lib() -> ctypes.CDLL:
                                   ctypes.POINTER(ctypes.c_double),
                                   ctypes.POINTER(ctypes.c_double)]),
         "kivi_status_string": (ctypes.c_char_p, [st]),
+        "kivi_decode_attention_static_scratch": (st, [ctypes.POINTER(KiviConfig), P, P, P, I32,
+                                                      I32, P, P, F32, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)

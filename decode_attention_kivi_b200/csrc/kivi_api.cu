@@ -3,8 +3,10 @@
 // here; the caller owns every buffer.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -277,8 +279,109 @@ const char* kivi_status_string(kivi_status status) {
     case KIVI_ERR_STATE: return "call not valid in the layer's current state";
     case KIVI_ERR_CUDA: return "CUDA runtime error";
     case KIVI_ERR_DEVICE: return "a kernel reported a failure in the device status word";
+    case KIVI_ERR_SCRATCH_LIMIT:
+      return "call needs more split-K scratch than KIVI_STATIC_SCRATCH_BYTES";
   }
   return "unknown status";
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode attention with a static scratch array, for callers that cannot
+// allocate device memory (see kivi_decode_attention_static_scratch in kivi.h).
+// ---------------------------------------------------------------------------
+
+// The split-K partials of kivi_decode_attention_static_scratch: the same layout
+// as a handle's workspace (header with the status word, then m/l, then acc).
+// In host code this name is only a stand-in for the device array; its device
+// address comes from cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_kivi_static_scratch[KIVI_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct StaticScratchSlot {
+  void* ptr = nullptr;  // device address of g_kivi_static_scratch on this device
+  int num_sms = 0;
+};
+
+std::mutex g_static_mu;
+StaticScratchSlot g_static_slots[kMaxDevices];
+
+// Once per device, with that device current: look up the array's address and
+// clear its header on `stream` (the status word must start at zero).
+kivi_status static_scratch_slot(cudaStream_t stream, StaticScratchSlot* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KIVI_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  StaticScratchSlot& slot = g_static_slots[dev];
+  if (slot.ptr == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_kivi_static_scratch) != cudaSuccess || p == nullptr)
+      return KIVI_ERR_CUDA;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return KIVI_ERR_CUDA;
+    if (cudaMemsetAsync(p, 0, kivi::kWsHeader, stream) != cudaSuccess) return KIVI_ERR_CUDA;
+    slot.ptr = p;
+    slot.num_sms = sms;
+  }
+  *out = slot;
+  return KIVI_OK;
+}
+
+}  // namespace
+
+extern "C" kivi_status kivi_decode_attention_static_scratch(
+    const kivi_config* cfg, const void* records, const void* resid_k, const void* resid_v,
+    int32_t layer, int32_t S, const void* q, float* out, float sm_scale, void* stream) {
+  kivi_status st = validate_config(cfg);
+  if (st != KIVI_OK) return st;
+  const int ngcap = kivi::num_groups(cfg->max_tokens);
+  if (layer < 0 || layer >= cfg->num_layers) return KIVI_ERR_INVALID_ARG;
+  if ((ngcap > 0 && !records) || !resid_k || !resid_v || !q || !out)
+    return KIVI_ERR_INVALID_ARG;
+  if ((records && !aligned16(records)) || !aligned16(resid_k) || !aligned16(resid_v) ||
+      !aligned16(q) || !aligned16(out))
+    return KIVI_ERR_INVALID_ARG;
+  if (!std::isfinite(sm_scale)) return KIVI_ERR_INVALID_ARG;
+  if (S < 0) return KIVI_ERR_INVALID_ARG;
+  if (S == 0) return KIVI_ERR_STATE;
+  if (S > cfg->max_tokens) return KIVI_ERR_CAPACITY;
+  const size_t rows = (size_t)cfg->batch * cfg->num_q_heads;
+  const size_t per_split = rows * (2 + (size_t)cfg->head_dim) * sizeof(float);
+  if (kivi::kWsHeader + per_split > KIVI_STATIC_SCRATCH_BYTES) return KIVI_ERR_SCRATCH_LIMIT;
+  const int fit = (int)((KIVI_STATIC_SCRATCH_BYTES - kivi::kWsHeader) / per_split);
+  const int max_splits = std::min(kivi::max_splits(cfg->batch, cfg->num_kv_heads), fit);
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  StaticScratchSlot slot;
+  st = static_scratch_slot(s, &slot);
+  if (st != KIVI_OK) return st;
+
+  const size_t seqs = (size_t)cfg->batch * cfg->num_kv_heads;
+  const long rb = record_bytes(cfg);
+  kivi::DecodeArgs a;
+  a.records = static_cast<const uint8_t*>(records) + (size_t)layer * seqs * ngcap * rb;
+  a.ring_k = static_cast<const __nv_bfloat16*>(resid_k) +
+             (size_t)layer * seqs * kRingSlots * cfg->head_dim;
+  a.ring_v = static_cast<const __nv_bfloat16*>(resid_v) +
+             (size_t)layer * seqs * kRingSlots * cfg->head_dim;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.out = out;
+  uint8_t* ws = static_cast<uint8_t*>(slot.ptr);
+  a.status = reinterpret_cast<uint32_t*>(ws);
+  a.ws_ml = reinterpret_cast<float*>(ws + kivi::kWsHeader);
+  a.ws_acc = a.ws_ml + 2 * rows * max_splits;
+  a.B = cfg->batch;
+  a.Hkv = cfg->num_kv_heads;
+  a.Hq = cfg->num_q_heads;
+  a.S = S;
+  a.ngcap = ngcap;
+  a.sm_scale = sm_scale;
+  a.max_splits = max_splits;
+  a.num_sms = slot.num_sms;
+  return from_cuda(kivi::launch_decode(cfg->head_dim, cfg->bits, a, s));
+}

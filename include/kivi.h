@@ -81,8 +81,14 @@ typedef enum {
   KIVI_ERR_CAPACITY = 4,         /* the call would exceed max_tokens */
   KIVI_ERR_STATE = 5,            /* prefill on a non-empty layer, append/attend on an empty one */
   KIVI_ERR_CUDA = 6,             /* a CUDA runtime call or launch failed */
-  KIVI_ERR_DEVICE = 7            /* a kernel reported a failure in the device status word */
+  KIVI_ERR_DEVICE = 7,           /* a kernel reported a failure in the device status word */
+  KIVI_ERR_SCRATCH_LIMIT = 8     /* the call needs more than the library's static scratch array */
 } kivi_status;
+
+/* Size of the file-scope device array used by
+ * kivi_decode_attention_static_scratch (every GPU that loads the library holds
+ * it until the process exits). */
+#define KIVI_STATIC_SCRATCH_BYTES (8u << 20)
 
 /* Cache geometry.  Supported: bits in {2, 4}, group_size == 32,
  * residual == 128, head_dim in {64, 128}, num_q_heads / num_kv_heads in
@@ -169,6 +175,31 @@ kivi_status kivi_append_token(kivi_cache* cache, int32_t layer,
 kivi_status kivi_decode_attention(const kivi_cache* cache, int32_t layer,
                                   const void* q, float* out, float sm_scale,
                                   void* stream);
+
+/* Decode attention that allocates nothing and needs neither a handle nor a
+ * workspace buffer.  The pages have no counterpart: this entry point is for
+ * callers that cannot allocate device memory - for example an inference engine
+ * that loads this library as a plugin and owns all device memory through its
+ * own pool allocator (a cudaMalloc behind its back would fail or break its
+ * accounting), or a process whose device memory is already reserved by such an
+ * allocator.  The caller passes only inputs and outputs: the cache buffers of
+ * `cfg` in the layout above (records may be NULL when NG(max_tokens) == 0),
+ * the layer, its token count S (for example from kivi_cache_length), q and
+ * out exactly as for kivi_decode_attention, whose result this call reproduces.
+ * Scratch: the split-K partials go to one file-scope device array of
+ * KIVI_STATIC_SCRATCH_BYTES.  The first call on a device looks up the array's
+ * address with cudaGetSymbolAddress and clears its header on `stream`; make
+ * that first call before any stream capture.  All calls on a device share the
+ * array and leave their contents in it: calls whose kernels may overlap on the
+ * GPU (other streams, other host threads) race on it and must be serialised by
+ * the caller.  The call picks at most as many splits as fit the array.
+ * Errors: INVALID_ARG, UNSUPPORTED, STATE (S == 0), CAPACITY (S > max_tokens),
+ * SCRATCH_LIMIT (one split's partials, 256 + B*Hq*(D+2)*4 bytes, exceed the
+ * array), CUDA. */
+kivi_status kivi_decode_attention_static_scratch(const kivi_config* cfg, const void* records,
+                                                 const void* resid_k, const void* resid_v,
+                                                 int32_t layer, int32_t S, const void* q,
+                                                 float* out, float sm_scale, void* stream);
 
 /* Synchronises `stream`, then reads and clears the device status word.
  * Returns KIVI_ERR_DEVICE if a kernel recorded a failure (a bounded wait that

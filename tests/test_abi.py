@@ -89,7 +89,7 @@ def test_null_handle_calls_fail_cleanly(lib):
 
 
 def test_status_strings(lib):
-    for code in range(8):
+    for code in range(9):
         assert lib.kivi_status_string(code)
     assert lib.kivi_status_string(99) == b"unknown status"
 

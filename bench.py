@@ -12,6 +12,7 @@ data-path collective); time = max over ranks.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -43,6 +44,8 @@ def parse():
     p.add_argument("--impl", default="kivi", choices=["kivi", "reference"])
     p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     p.add_argument("--batch", type=int, default=None, help="override the workload's batch")
+    p.add_argument("--layers", type=int, default=None,
+                   help="override the workload's layer count (small profiling captures)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     return p.parse_args()
@@ -386,6 +389,8 @@ def main():
     w = synth.WORKLOADS[args.workload]
     if args.batch:
         w = w.with_batch(args.batch)
+    if args.layers:
+        w = dataclasses.replace(w, num_layers=args.layers)
     if args.impl == "reference":
         if rank == 0:
             run_reference(args, w)

@@ -352,7 +352,9 @@ extern "C" kivi_status kivi_decode_attention_static_scratch(
   if (S > cfg->max_tokens) return KIVI_ERR_CAPACITY;
   const size_t rows = (size_t)cfg->batch * cfg->num_q_heads;
   const size_t per_split = rows * (2 + (size_t)cfg->head_dim) * sizeof(float);
-  if (kivi::kWsHeader + per_split > KIVI_STATIC_SCRATCH_BYTES) return KIVI_ERR_SCRATCH_LIMIT;
+  // at least one split over the quantized groups plus the residual chunks
+  if (kivi::kWsHeader + kivi::kMinSplits * per_split > KIVI_STATIC_SCRATCH_BYTES)
+    return KIVI_ERR_SCRATCH_LIMIT;
   const int fit = (int)((KIVI_STATIC_SCRATCH_BYTES - kivi::kWsHeader) / per_split);
   const int max_splits = std::min(kivi::max_splits(cfg->batch, cfg->num_kv_heads), fit);
 

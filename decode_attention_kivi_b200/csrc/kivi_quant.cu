@@ -28,10 +28,8 @@ struct QuantSmem {
   uint8_t vc[kGroup][D];
 };
 
-__device__ __forceinline__ uint32_t pack_meta(float scale, float mn) {
-  const uint32_t s = __half_as_ushort(__float2half_rn(scale));
-  const uint32_t m = __half_as_ushort(__float2half_rn(mn));
-  return s | (m << 16);
+__device__ __forceinline__ unsigned short to_f16_bits(float x) {
+  return __half_as_ushort(__float2half_rn(x));
 }
 
 // Codes of one group of values already reduced to (mn, scale).
@@ -61,8 +59,11 @@ __device__ void quantize_tiles_to_record(QuantSmem<D>& sm, uint32_t* __restrict_
   constexpr RecordGeom geo{D, BITS};
   constexpr int kQmax = (1 << BITS) - 1;
   constexpr int kCpw = geo.codes_per_word();
-  uint32_t* kmeta = rec + geo.k_meta_off() / 4;
-  uint32_t* vmeta = rec + geo.v_meta_off() / 4;
+  unsigned short* rec16 = reinterpret_cast<unsigned short*>(rec);
+  unsigned short* kscale = rec16 + geo.k_scale_off() / 2;
+  unsigned short* kmin = rec16 + geo.k_min_off() / 2;
+  unsigned short* vscale = rec16 + geo.v_scale_off() / 2;
+  unsigned short* vmin = rec16 + geo.v_min_off() / 2;
   // Keys: per channel d over the 32 tokens.
   for (int d = threadIdx.x; d < D; d += kQuantThreads) {
     float mn = __bfloat162float(sm.k[0][d]), mx = mn;
@@ -75,7 +76,8 @@ __device__ void quantize_tiles_to_record(QuantSmem<D>& sm, uint32_t* __restrict_
     const float scale = __fdiv_rn(__fsub_rn(mx, mn), (float)kQmax);
 #pragma unroll 8
     for (int t = 0; t < kGroup; ++t) sm.kc[t][d] = quant_code<BITS>(__bfloat162float(sm.k[t][d]), mn, scale);
-    kmeta[d] = pack_meta(scale, mn);
+    kscale[d] = to_f16_bits(scale);
+    kmin[d] = to_f16_bits(mn);
   }
   // Values: per token t over channel block j.
   constexpr int kBlocks = D / 32;
@@ -92,7 +94,8 @@ __device__ void quantize_tiles_to_record(QuantSmem<D>& sm, uint32_t* __restrict_
 #pragma unroll 8
     for (int c = 0; c < 32; ++c)
       sm.vc[t][32 * j + c] = quant_code<BITS>(__bfloat162float(sm.v[t][32 * j + c]), mn, scale);
-    vmeta[t * kBlocks + j] = pack_meta(scale, mn);
+    vscale[v_meta_index(t, j)] = to_f16_bits(scale);
+    vmin[v_meta_index(t, j)] = to_f16_bits(mn);
   }
   __syncthreads();
   // Pack: K token-major rows (channels innermost), V channel-major rows (tokens innermost).
@@ -101,14 +104,27 @@ __device__ void quantize_tiles_to_record(QuantSmem<D>& sm, uint32_t* __restrict_
     const int t = wi / geo.k_row_words(), w = wi % geo.k_row_words();
     uint32_t word = 0;
 #pragma unroll
-    for (int i = 0; i < kCpw; ++i) word |= (uint32_t)sm.kc[t][w * kCpw + i] << (i * BITS);
+    for (int i = 0; i < kCpw; ++i) word |= (uint32_t)sm.kc[t][w * kCpw + i] << code_bit(i, BITS);
     rec[wi] = word;
   }
+  // V: word wi belongs to (g, tig, mt) = its block of BITS/2 words; each word
+  // holds 16/BITS pairs idx = 4kk + 2hf + r of tokens 16kk+8hf+2tig+{0,1} of
+  // channel 16mt+g+8r (inverse of v_code_word / v_code_bit).
+  constexpr int kWordsPer = BITS / 2, kPairs = 16 / BITS;
   for (int wi = threadIdx.x; wi < kWords; wi += kQuantThreads) {
-    const int d = wi / geo.v_row_words(), w = wi % geo.v_row_words();
+    const int base = wi / kWordsPer, w2 = wi % kWordsPer;
+    const int mt = base % (D / 16), gt = base / (D / 16);
+    const int g = gt / 4, tig = gt % 4;
     uint32_t word = 0;
 #pragma unroll
-    for (int i = 0; i < kCpw; ++i) word |= (uint32_t)sm.vc[w * kCpw + i][d] << (i * BITS);
+    for (int p = 0; p < kPairs; ++p) {
+      const int idx = w2 * kPairs + p;
+      const int kk = idx / 4, hf = (idx / 2) % 2, r = idx % 2;
+      const int d = 16 * mt + g + 8 * r;
+      const int t0 = 16 * kk + 8 * hf + 2 * tig;
+      word |= (uint32_t)sm.vc[t0][d] << (p * BITS);
+      word |= (uint32_t)sm.vc[t0 + 1][d] << (16 + p * BITS);
+    }
     rec[geo.v_codes_off() / 4 + wi] = word;
   }
 }

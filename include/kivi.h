@@ -35,16 +35,22 @@
  *   records  [L][B][Hkv][NGcap] group records, NGcap = NG(max_tokens),
  *            record bytes = G*D*b/4 + 8*D (3072 at D=128 b=2, 5120 at b=4,
  *            1536 at D=64 b=2).  One record, in order:
- *     K codes  G rows (token i of the group) x D*b/32 words; the code of
- *              channel d sits at bit (d mod (32/b))*b of word d/(32/b).
- *     V codes  D rows (channel d) x G*b/32 words; the code of token i sits at
- *              bit (i mod (32/b))*b of word i/(32/b).  Each code array is
- *              stored with the axis its attention product sums over innermost
- *              (channels for q.k, tokens for p.v).
- *     K meta   D entries {fp16 scale, fp16 min} (scale at the lower address),
- *              entry d = channel d.
- *     V meta   G * (D/32) entries {fp16 scale, fp16 min}, entry i*(D/32) + j =
- *              token i, channels [32j, 32j + 32).
+ *     K codes  G rows (token i of the group) x D*b/32 words; channel d is code
+ *              n = d mod (32/b) of word d/(32/b), at bit (n mod 2)*16 + (n/2)*b
+ *              (even codes in the low 16 bits, odd codes in the high 16 bits).
+ *     V codes  G*D*b/32 words in the order the decode kernel's threads consume
+ *              them.  Token i, channel d: with mt = d/16, g = d mod 8,
+ *              r = (d mod 16)/8, kk = i/16, hf = (i mod 16)/8, tig = (i mod 8)/2,
+ *              e = i mod 2, idx = 4kk + 2hf + r and p = 16/b:
+ *                word = ((4g + tig)*(D/16) + mt)*(b/2) + idx/p,
+ *                bit  = 16e + (idx mod p)*b.
+ *     K scale  D fp16 (channel d), then K min: D fp16.
+ *     V scale  (D/32) blocks of G fp16; token i of block j at index
+ *              32j + 2(4tig + 2kk + hf) + e (tig, kk, hf, e of i as above);
+ *              then V min in the same layout.
+ *              Each array puts the operands one thread reads next to each
+ *              other, so the kernel turns a pair of codes into an fp16x2
+ *              register with one mask-and-or.
  *   resid_k, resid_v  bf16 [L][B][Hkv][R + G][D].
  *
  * Conventions for every call below:
@@ -92,9 +98,10 @@ typedef enum {
 
 /* Cache geometry.  Supported: bits in {2, 4}, group_size == 32,
  * residual == 128, head_dim in {64, 128}, num_q_heads / num_kv_heads in
- * {1, 2, 4, 8} (exact multiple), all counts >= 1, max_tokens >= 1.  Query head h reads kv head h / (num_q_heads / num_kv_heads)
- * (consecutive grouping, the usual repeat-KV convention; [Llama-3 rec] "Model"
- * gives 32 query heads over 8 kv heads). */
+ * {1, 2, 4, 8} (exact multiple), all counts >= 1, max_tokens >= 1.  Query
+ * head h reads kv head h / (num_q_heads / num_kv_heads) (consecutive grouping,
+ * the usual repeat-KV convention; [Llama-3 rec] "Model" gives 32 query heads
+ * over 8 kv heads). */
 typedef struct {
   int32_t batch;
   int32_t num_layers;
@@ -194,8 +201,9 @@ kivi_status kivi_decode_attention(const kivi_cache* cache, int32_t layer,
  * GPU (other streams, other host threads) race on it and must be serialised by
  * the caller.  The call picks at most as many splits as fit the array.
  * Errors: INVALID_ARG, UNSUPPORTED, STATE (S == 0), CAPACITY (S > max_tokens),
- * SCRATCH_LIMIT (one split's partials, 256 + B*Hq*(D+2)*4 bytes, exceed the
- * array), CUDA. */
+ * SCRATCH_LIMIT (the partials of the fewest splits a call uses - one over the
+ * quantized groups and one per residual chunk of 32 tokens, 6 in all -
+ * 256 + 6*B*Hq*(D+2)*4 bytes, exceed the array), CUDA. */
 kivi_status kivi_decode_attention_static_scratch(const kivi_config* cfg, const void* records,
                                                  const void* resid_k, const void* resid_v,
                                                  int32_t layer, int32_t S, const void* q,

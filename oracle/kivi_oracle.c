@@ -136,9 +136,42 @@ int oracle_num_groups(int S) {
   return (S - ORACLE_R) / ORACLE_G;
 }
 
+/* Code `index` of a row goes to word index / (32/b); inside the word the
+ * even-indexed codes fill the low 16 bits and the odd-indexed codes the high 16
+ * bits, each half from its least significant bit: bit offset
+ * (index mod 2) * 16 + ((index mod (32/b)) / 2) * b. */
+static int code_bit_offset(int index, int bits) {
+  int in_word = index % (32 / bits);
+  return (in_word % 2) * 16 + (in_word / 2) * bits;
+}
+
 static void put_code(uint32_t* words, int index, int bits, int code) {
-  int per_word = 32 / bits;
-  words[index / per_word] |= (uint32_t)code << ((index % per_word) * bits);
+  words[index / (32 / bits)] |= (uint32_t)code << code_bit_offset(index, bits);
+}
+
+/* Value codes are stored in the order the decode kernel's threads consume
+ * them.  For token i (0..31) and channel d of a group record:
+ *   mt = d / 16, g = d mod 8, r = (d mod 16) / 8,
+ *   kk = i / 16, hf = (i mod 16) / 8, tig = (i mod 8) / 2, e = i mod 2,
+ *   idx = 4 kk + 2 hf + r, p = 16 / b pairs per word,
+ *   word = ((4 g + tig) * (D / 16) + mt) * (b / 2) + idx / p,
+ *   bit  = 16 e + (idx mod p) * b.
+ * So each word holds, for channels d and d + 8, pairs of adjacent tokens with
+ * the even token in the low 16 bits and the odd token in the high 16 bits. */
+static void v_code_position(int i, int d, int D, int bits, long* word, int* bit) {
+  const int mt = d / 16, g = d % 8, r = (d % 16) / 8;
+  const int kk = i / 16, hf = (i % 16) / 8, tig = (i % 8) / 2, e = i % 2;
+  const int idx = 4 * kk + 2 * hf + r, per_word = 16 / bits;
+  *word = ((long)(4 * g + tig) * (D / 16) + mt) * (bits / 2) + idx / per_word;
+  *bit = 16 * e + (idx % per_word) * bits;
+}
+
+/* fp16 index of the value scale (and min) of token i, channel block j: each
+ * block holds 16 token pairs, pair q = 4 tig + 2 kk + hf at indices 2q, 2q+1
+ * (with tig, kk, hf, e of token i as above). */
+static long v_meta_index(int i, int j) {
+  const int kk = i / 16, hf = (i % 16) / 8, tig = (i % 8) / 2, e = i % 2;
+  return (long)j * 32 + 2 * (4 * tig + 2 * kk + hf) + e;
 }
 
 static void put_u16(uint8_t* p, uint16_t v) {
@@ -161,8 +194,12 @@ void oracle_make_record(const uint16_t* k, const uint16_t* v, long ld, int D,
   uint32_t* vcodes = (uint32_t*)malloc(sizeof(uint32_t) * kc_words);
   memset(kcodes, 0, sizeof(uint32_t) * kc_words);
   memset(vcodes, 0, sizeof(uint32_t) * kc_words);
-  uint8_t* kmeta = record + 8L * kc_words;
-  uint8_t* vmeta = kmeta + 4L * D;
+  /* K meta: D fp16 scales, then D fp16 mins.  V meta: (D/32) x 32 fp16 scales
+   * (block j, then token i), then the same for the mins. */
+  uint8_t* kscale = record + 8L * kc_words;
+  uint8_t* kmin = kscale + 2L * D;
+  uint8_t* vscale = kmin + 2L * D;
+  uint8_t* vmin = vscale + 2L * D;
 
   float col[ORACLE_G];
   uint8_t codes[ORACLE_G];
@@ -173,8 +210,8 @@ void oracle_make_record(const uint16_t* k, const uint16_t* v, long ld, int D,
     oracle_quantize_group(col, G, 1, bits, &scale, &mn, codes);
     /* token-major rows of D*b/32 words: channel d of token i */
     for (int i = 0; i < G; ++i) put_code(kcodes + (long)i * D * bits / 32, d, bits, codes[i]);
-    put_u16(kmeta + 4L * d, oracle_f32_to_f16_bits(scale));
-    put_u16(kmeta + 4L * d + 2, oracle_f32_to_f16_bits(mn));
+    put_u16(kscale + 2L * d, oracle_f32_to_f16_bits(scale));
+    put_u16(kmin + 2L * d, oracle_f32_to_f16_bits(mn));
   }
   /* Values, per token i over channel block j. */
   float row[32];
@@ -183,12 +220,15 @@ void oracle_make_record(const uint16_t* k, const uint16_t* v, long ld, int D,
       for (int c = 0; c < 32; ++c) row[c] = bf16_bits_to_float(v[(long)i * ld + 32 * j + c]);
       float scale, mn;
       oracle_quantize_group(row, 32, 1, bits, &scale, &mn, codes);
-      /* channel-major rows of G*b/32 words: token i of channel 32j+c */
-      for (int c = 0; c < 32; ++c)
-        put_code(vcodes + (long)(32 * j + c) * G * bits / 32, i, bits, codes[c]);
-      long e = (long)i * (D / 32) + j;
-      put_u16(vmeta + 4 * e, oracle_f32_to_f16_bits(scale));
-      put_u16(vmeta + 4 * e + 2, oracle_f32_to_f16_bits(mn));
+      for (int c = 0; c < 32; ++c) {
+        long word;
+        int bit;
+        v_code_position(i, 32 * j + c, D, bits, &word, &bit);
+        vcodes[word] |= (uint32_t)codes[c] << bit;
+      }
+      const long e = v_meta_index(i, j);
+      put_u16(vscale + 2 * e, oracle_f32_to_f16_bits(scale));
+      put_u16(vmin + 2 * e, oracle_f32_to_f16_bits(mn));
     }
   }
   for (long w = 0; w < kc_words; ++w) {
@@ -207,7 +247,7 @@ static int get_code(const uint8_t* row, int index, int bits) {
   const uint8_t* w = row + 4L * (index / per_word);
   uint32_t word = (uint32_t)w[0] | ((uint32_t)w[1] << 8) | ((uint32_t)w[2] << 16) |
                   ((uint32_t)w[3] << 24);
-  return (int)((word >> ((index % per_word) * bits)) & ((1u << bits) - 1u));
+  return (int)((word >> code_bit_offset(index, bits)) & ((1u << bits) - 1u));
 }
 
 static uint16_t get_u16(const uint8_t* p) { return (uint16_t)(p[0] | (p[1] << 8)); }
@@ -218,20 +258,27 @@ void oracle_dequant_record(const uint8_t* record, int D, int bits, double* k_hat
                            double* v_hat) {
   const int G = ORACLE_G;
   const long row_words_k = (long)D * bits / 32;
-  const long row_words_v = (long)G * bits / 32;
   const long kc_bytes = 4L * G * row_words_k;
-  const uint8_t* kmeta = record + 2 * kc_bytes;
-  const uint8_t* vmeta = kmeta + 4L * D;
+  const uint8_t* kscale = record + 2 * kc_bytes;
+  const uint8_t* kmin = kscale + 2L * D;
+  const uint8_t* vscale = kmin + 2L * D;
+  const uint8_t* vmin = vscale + 2L * D;
   for (int i = 0; i < G; ++i) {
     for (int d = 0; d < D; ++d) {
       int ck = get_code(record + 4L * row_words_k * i, d, bits);
-      double sk = oracle_f16_bits_to_double(get_u16(kmeta + 4L * d));
-      double mk = oracle_f16_bits_to_double(get_u16(kmeta + 4L * d + 2));
+      double sk = oracle_f16_bits_to_double(get_u16(kscale + 2L * d));
+      double mk = oracle_f16_bits_to_double(get_u16(kmin + 2L * d));
       k_hat[(long)i * D + d] = sk * ck + mk;
-      int cv = get_code(record + kc_bytes + 4L * row_words_v * d, i, bits);
-      long e = (long)i * (D / 32) + d / 32;
-      double sv = oracle_f16_bits_to_double(get_u16(vmeta + 4 * e));
-      double mv = oracle_f16_bits_to_double(get_u16(vmeta + 4 * e + 2));
+      long vw;
+      int vb;
+      v_code_position(i, d, D, bits, &vw, &vb);
+      const uint8_t* wp = record + kc_bytes + 4 * vw;
+      const uint32_t vword = (uint32_t)wp[0] | ((uint32_t)wp[1] << 8) |
+                             ((uint32_t)wp[2] << 16) | ((uint32_t)wp[3] << 24);
+      int cv = (int)((vword >> vb) & ((1u << bits) - 1u));
+      long e = v_meta_index(i, d / 32);
+      double sv = oracle_f16_bits_to_double(get_u16(vscale + 2 * e));
+      double mv = oracle_f16_bits_to_double(get_u16(vmin + 2 * e));
       v_hat[(long)i * D + d] = sv * cv + mv;
     }
   }

@@ -161,18 +161,43 @@ def test_packed_words_hand_worked(bits):
     if bits == 2:
         assert _word(rec, 0) == int(g["2bit_k_row0_word0"], 16)
         assert _word(rec, row_bytes_k) == int(g["2bit_k_row1_word0"], 16)
-        vbase = 32 * row_bytes_k
-        row_bytes_v = 32 * bits // 8
-        assert _word(rec, vbase) == int(g["2bit_v_chan0_word0"], 16)
-        assert _word(rec, vbase + row_bytes_v) == int(g["2bit_v_chan1_word0"], 16)
     else:
         assert _word(rec, 0) == int(g["4bit_k_row0_word0"], 16)
         assert _word(rec, 4) == int(g["4bit_k_row0_word1"], 16)
         assert _word(rec, row_bytes_k) == int(g["4bit_k_row1_word0"], 16)
-    kmeta = 2 * 32 * row_bytes_k
-    assert list(rec[kmeta:kmeta + 4]) == g["meta_scale1_min0_bytes"]
-    vmeta = kmeta + 4 * D
-    assert list(rec[vmeta:vmeta + 4]) == g["meta_scale1_min0_bytes"]
+    kscale = 2 * 32 * row_bytes_k
+    kmin, vscale = kscale + 2 * D, kscale + 4 * D
+    vmin = vscale + 2 * D
+    assert list(rec[kscale:kscale + 2]) == g["fp16_one_bytes"]
+    assert list(rec[kmin:kmin + 2]) == g["fp16_zero_bytes"]
+    assert list(rec[vscale:vscale + 2]) == g["fp16_one_bytes"]
+    assert list(rec[vmin:vmin + 2]) == g["fp16_zero_bytes"]
+    assert len(rec) == vmin + 2 * D
+    k_hat, v_hat = O.dequant_record(rec, D, bits)
+    assert np.array_equal(k_hat, tile) and np.array_equal(v_hat, tile)
+
+
+@pytest.mark.parametrize("case", range(4))
+def test_one_hot_positions_hand_worked(case):
+    """A single non-zero code lands at the word, bit and metadata slot the layout
+    definition gives (positions worked by hand in tests/golden/hand_worked.json)."""
+    c = _golden("hand_worked.json")["one_hot"]["cases"][case]
+    bits, i, d, D = c["bits"], c["i"], c["d"], 128
+    tile = np.zeros((32, D), np.float32)
+    tile[i, d] = (1 << bits) - 1
+    tb = _bits(torch.tensor(tile))
+    rec = O.make_record(tb, tb, bits)
+    words = rec[:len(rec) - 8 * D].view("<u4")
+    n_k = 32 * D * bits // 32
+    kw, vw = words[:n_k], words[n_k:2 * n_k]
+    assert np.count_nonzero(kw) == 1 and kw[c["k_word"]] == int(c["k_value"], 16)
+    assert np.count_nonzero(vw) == 1 and vw[c["v_word"]] == int(c["v_value"], 16)
+    meta = rec[len(rec) - 8 * D:].view("<u2")
+    kscale, kmin, vscale, vmin = meta[:D], meta[D:2 * D], meta[2 * D:3 * D], meta[3 * D:]
+    one = 0x3C00
+    assert np.count_nonzero(kscale) == 1 and kscale[c["k_scale_f16_index"]] == one
+    assert np.count_nonzero(vscale) == 1 and vscale[c["v_scale_f16_index"]] == one
+    assert not kmin.any() and not vmin.any()
     k_hat, v_hat = O.dequant_record(rec, D, bits)
     assert np.array_equal(k_hat, tile) and np.array_equal(v_hat, tile)
 

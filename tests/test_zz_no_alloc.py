@@ -68,12 +68,13 @@ def test_static_scratch_matches_workspace_entry_point(kivi):
 
 
 def test_static_scratch_rejects_oversized_calls(kivi):
-    """One split's partials above the array's size is refused before any launch."""
+    """A call whose fewest splits (one over the groups, five residual chunks) do not fit
+    the array is refused before any launch."""
     from decode_attention_kivi_b200 import _native as N
 
     cfg = kivi.make_config(batch=512, num_layers=1, num_kv_heads=64, num_q_heads=64,
                            head_dim=128, bits=2, max_tokens=4096)
-    assert 256 + 512 * 64 * 130 * 4 > N.STATIC_SCRATCH_BYTES
+    assert 256 + 6 * 512 * 64 * 130 * 4 > N.STATIC_SCRATCH_BYTES
     fake = 1 << 20
     rc = N.lib().kivi_decode_attention_static_scratch(ctypes.byref(cfg), fake, fake, fake, 0,
                                                       300, fake, fake, 0.0, None)

@@ -68,6 +68,19 @@ def attention_bytes(w: synth.Workload, S: int) -> int:
             + w.batch * w.num_q_heads * w.head_dim * (2 + 4))
 
 
+def max_over_ranks(values, device) -> list:
+    """Element-wise max of per-rank timings over the process group (any backend)."""
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if torch.distributed.is_initialized() and torch.distributed.get_world_size() > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def weak_scaling_tokens_per_s(world: int, batch: int, steps: int, ms: float) -> float:
+    """Whole-job decode throughput: every rank decodes its own batch for `steps` steps."""
+    return world * batch * steps / (ms * 1e-3)
+
+
 def workload_config(w: synth.Workload, s_first: int, s_last: int, l2_note: str) -> dict:
     return {"workload": w.name, "batch_per_gpu": w.batch, "layers": w.num_layers,
             "kv_heads": w.num_kv_heads, "q_heads": w.num_q_heads, "head_dim": w.head_dim,
@@ -249,13 +262,9 @@ def run_gpu(args, w: synth.Workload, rank: int, world: int):
         e2e = run_e2e(args, w, cache, L, h, sptr, device, world)
 
     if world > 1:
-        t = torch.tensor([ms, attn_ms], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms, attn_ms = float(t[0]), float(t[1])
+        ms, attn_ms = max_over_ranks([ms, attn_ms], device)
         if e2e is not None:
-            te = torch.tensor([e2e["_ms"]], device=device, dtype=torch.float64)
-            torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
-            e2e["_ms"] = float(te[0])
+            e2e["_ms"] = max_over_ranks([e2e["_ms"]], device)[0]
     cache.close()
     return dict(ms=ms, attn_ms=attn_ms, n_attn=n_attn, bytes_timed=bytes_timed,
                 s_first=s_first, s_last=s_last, clocks=clocks, e2e=e2e)
@@ -408,7 +417,7 @@ def main():
         peak, peak_kind = hbm_peak()
         gbs = res["bytes_timed"] / (res["attn_ms"] * 1e-3) / 1e9
         per_launch = res["bytes_timed"] / res["n_attn"]
-        value = world * w.batch * args.steps / (res["ms"] * 1e-3)
+        value = weak_scaling_tokens_per_s(world, w.batch, args.steps, res["ms"])
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms"] / args.steps,
@@ -428,7 +437,7 @@ def main():
         }
         if res["e2e"] is not None:
             e = res["e2e"]
-            line["e2e"] = {"value": world * w.batch * args.steps / (e["_ms"] * 1e-3),
+            line["e2e"] = {"value": weak_scaling_tokens_per_s(world, w.batch, args.steps, e["_ms"]),
                            "unit": "tokens/s", "h2d_bytes_per_step": e["h2d_bytes_per_step"],
                            "d2h_bytes_per_step": e["d2h_bytes_per_step"]}
         if world == 1 and not args.no_cpu_baseline:

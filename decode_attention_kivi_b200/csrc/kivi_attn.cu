@@ -33,6 +33,7 @@
 #include <cuda_fp16.h>
 
 #include "kivi_kernels.h"
+#include "kivi_launch.cuh"
 #include "kivi_layout.cuh"
 
 namespace kivi {
@@ -261,6 +262,7 @@ decode_kernel(DecodeArgs args, int splits_g, int n_res, int groups_per_cta, floa
   const long seq = (long)b * args.Hkv + kvh;
   const int NG = num_groups(S);
 
+  wait_for_predecessor();  // q, the records and the rings may come from the previous kernel
   // q of this kv head's query heads, fp32 in smem; per-head exponent e_h with
   // max |q_h| * 2^-e_h in [0.5, 1).
   for (int i = threadIdx.x; i < HPK * D; i += kThreads) {
@@ -662,6 +664,7 @@ decode_kernel(DecodeArgs args, int splits_g, int n_res, int groups_per_cta, floa
     // a chunk starts at a multiple of 32 tokens, so its ring slots are
     // contiguous), then scores, the chunk softmax and P.V read shared memory.
     // This CTA writes its partial directly and returns.
+    allow_successor();
     const int chunk = split - splits_g;
     const int t0 = NG * kGroup + chunk * kGroup;
     const int n = min(kGroup, S - t0);
@@ -736,6 +739,7 @@ decode_kernel(DecodeArgs args, int splits_g, int n_res, int groups_per_cta, floa
     return;
   }
 
+  allow_successor();
   // ===================== merge the warps, write this CTA's partial =====================
   __syncthreads();
   const int splits_total = splits_g + n_res;
@@ -767,6 +771,8 @@ decode_kernel(DecodeArgs args, int splits_g, int n_res, int groups_per_cta, floa
 // out[b][h] = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s.
 template <int D>
 __global__ void __launch_bounds__(D) combine_kernel(DecodeArgs args, int splits) {
+  wait_for_predecessor();  // every split's partial is written
+  allow_successor();
   const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
   const long part0 = ((long)b * args.Hq + h) * splits;
   float M = -INFINITY;
@@ -807,10 +813,11 @@ cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t stream) {
   const int r = a.S - NG * kGroup;                      // residual tokens, >= 1
   const int n_res = (r + kGroup - 1) / kGroup;           // residual chunks, <= 5
   const int n_ctas = (splits_g + n_res) * a.Hkv * a.B;
-  decode_kernel<D, BITS, HPK><<<n_ctas, kThreads, P::kBytes, stream>>>(a, splits_g, n_res, gpc,
-                                                                       qscale);
-  dim3 cgrid(a.Hq, a.B);
-  combine_kernel<D><<<cgrid, D, 0, stream>>>(a, splits_g + n_res);
+  cudaError_t e = launch_pdl(decode_kernel<D, BITS, HPK>, dim3(n_ctas), dim3(kThreads), P::kBytes,
+                             stream, a, splits_g, n_res, gpc, qscale);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(combine_kernel<D>, dim3(a.Hq, a.B), dim3(D), 0, stream, a, splits_g + n_res);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -1,0 +1,43 @@
+// kivi_launch.cuh - programmatic dependent launch (PDL) for the per-step kernels.
+//
+// append -> decode -> combine -> (next layer's) append run back to back on one
+// stream.  Launching each with programmatic stream serialization lets the GPU
+// schedule a kernel's CTAs while its predecessor drains; every kernel executes
+// griddepcontrol.wait before it touches memory the predecessor may write, so
+// the stream's ordering guarantees are unchanged.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <utility>
+
+namespace kivi {
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// Waits until the preceding kernel on the stream has completed and its writes
+// are visible (a no-op when the launch was not programmatic).
+__device__ __forceinline__ void wait_for_predecessor() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Allows the next kernel on the stream to begin launching its CTAs.
+__device__ __forceinline__ void allow_successor() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+}  // namespace kivi

@@ -13,6 +13,7 @@
 #include <cuda_fp16.h>
 
 #include "kivi_kernels.h"
+#include "kivi_launch.cuh"
 #include "kivi_layout.cuh"
 
 namespace kivi {
@@ -175,6 +176,8 @@ append_kernel(const __nv_bfloat16* __restrict__ k_new, const __nv_bfloat16* __re
   __shared__ __align__(16) QuantSmem<D> sm;
   constexpr RecordGeom geo{D, BITS};
   constexpr int kVecPerRow = D * 2 / 16;
+  wait_for_predecessor();  // the previous kernel may still read this layer's ring
+  allow_successor();
   const int h = blockIdx.x, b = blockIdx.y;
   const long seq = (long)b * Hkv + h;
   __nv_bfloat16* rk = ring_k + seq * kRingSlots * D;
@@ -217,9 +220,10 @@ cudaError_t launch_prefill_t(const PrefillArgs& a, cudaStream_t stream) {
 template <int D, int BITS>
 cudaError_t launch_append_t(const AppendArgs& a, cudaStream_t stream) {
   dim3 grid(a.Hkv, a.B);
-  append_kernel<D, BITS><<<grid, kQuantThreads, 0, stream>>>(a.k_new, a.v_new, a.S, a.Hkv,
-                                                            a.ngcap, a.flush, a.ng, a.ring_k,
-                                                            a.ring_v, a.records);
+  cudaError_t e = launch_pdl(append_kernel<D, BITS>, grid, dim3(kQuantThreads), 0, stream,
+                             a.k_new, a.v_new, a.S, a.Hkv, a.ngcap, a.flush, a.ng, a.ring_k,
+                             a.ring_v, a.records);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

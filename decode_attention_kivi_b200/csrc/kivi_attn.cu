@@ -167,11 +167,20 @@ __device__ __forceinline__ uint32_t hadd2(uint32_t a, uint32_t b) {
   return d;
 }
 
+// (w & mask) | magic as one three-input logic op (LUT 0xEA = (a & b) | c); the
+// two-operator C form costs two instructions.
+template <uint32_t MASK>
+__device__ __forceinline__ uint32_t and_or(uint32_t w, uint32_t magic) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(w), "n"(MASK), "r"(magic));
+  return d;
+}
+
 template <int BITS, int P>
 __device__ __forceinline__ uint32_t code_pair(uint32_t w, const CodeConsts<BITS>& k) {
   static_assert(P + BITS <= 10 && P % BITS == 0, "code bits must lie inside the fp16 mantissa");
   constexpr uint32_t m = ((1u << BITS) - 1u) << P;
-  return hadd2((w & (m | (m << 16))) | k.magic[P / BITS], k.neg[P / BITS]);
+  return hadd2(and_or<m | (m << 16)>(w, k.magic[P / BITS]), k.neg[P / BITS]);
 }
 
 // Pair K (codes 2K and 2K+1) of a word; pairs past the fp16 mantissa come from
@@ -225,7 +234,7 @@ struct Plan {
 // ---------------------------------------------------------------------------
 
 template <int D, int BITS, int HPK>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, HPK <= 4 ? 4 : 2)
 decode_kernel(DecodeArgs args, int splits_g, int n_res, int groups_per_cta, float qscale) {
   // Linear grid: B*Hkv*splits_g group CTAs (split fastest), then B*Hkv*n_res
   // residual-chunk CTAs, so the short residual CTAs run last and fill the tail.
@@ -270,7 +279,7 @@ decode_kernel(DecodeArgs args, int splits_g, int n_res, int groups_per_cta, floa
     q_s[i] = __bfloat162float(args.q[((long)b * Hq + kvh * HPK + hh) * D + d]);
   }
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 0 && split < splits_g) {  // the residual CTAs do not scale q
     for (int hh = 0; hh < HPK; ++hh) {
       float mx = 0.f;
       for (int d = lane; d < D; d += 32) mx = fmaxf(mx, fabsf(q_s[hh * D + d]));
@@ -675,12 +684,27 @@ decode_kernel(DecodeArgs args, int splits_g, int n_res, int groups_per_cta, floa
     static_assert(2 * kGroup * D * 2 + HPK * kGroup * 4 <= P::kStageBytes,
                   "residual chunk must fit in the stage area");
     {
+      // every load of the chunk is issued before the first store: one round trip
       const uint4* gk = reinterpret_cast<const uint4*>(args.ring_k + (seq * kRingSlots + slot0) * D);
       const uint4* gv = reinterpret_cast<const uint4*>(args.ring_v + (seq * kRingSlots + slot0) * D);
       const int n16 = n * D * 2 / 16;
-      for (int i = threadIdx.x; i < n16; i += kThreads) {
-        reinterpret_cast<uint4*>(kc)[i] = gk[i];
-        reinterpret_cast<uint4*>(vc)[i] = gv[i];
+      constexpr int kPer = (kGroup * D * 2 / 16 + kThreads - 1) / kThreads;
+      uint4 rk[kPer], rv[kPer];
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) {
+        const int i = threadIdx.x + k * kThreads;
+        if (i < n16) {
+          rk[k] = gk[i];
+          rv[k] = gv[i];
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) {
+        const int i = threadIdx.x + k * kThreads;
+        if (i < n16) {
+          reinterpret_cast<uint4*>(kc)[i] = rk[k];
+          reinterpret_cast<uint4*>(vc)[i] = rv[k];
+        }
       }
     }
     __syncthreads();
@@ -791,18 +815,27 @@ __global__ void __launch_bounds__(D) combine_kernel(DecodeArgs args, int splits)
 template <int D, int BITS, int HPK>
 cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t stream) {
   using P = Plan<D, BITS, HPK>;
-  static bool attr_set = false;  // per process; every device gets the same attribute
-  if (!attr_set) {
+  // Per process (every device of a process is the same part): the largest
+  // shared-memory carveout, and the CTAs per SM that the kernel really gets.
+  static int ctas_per_sm = 0;
+  if (ctas_per_sm == 0) {
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, BITS, HPK>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, P::kBytes);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    e = cudaFuncSetAttribute(decode_kernel<D, BITS, HPK>,
+                             cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    int n = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<D, BITS, HPK>, kThreads,
+                                                      P::kBytes);
+    if (e != cudaSuccess) return e;
+    ctas_per_sm = max(1, n);
   }
   const int NG = num_groups(a.S);
   const int pairs = a.B * a.Hkv;
   int splits_g = 0, gpc = 1;
   if (NG > 0) {
-    const int ctas_per_sm = P::kBytes <= 56 * 1024 ? 4 : 2;
     const int want = max(1, (a.num_sms * ctas_per_sm) / pairs);   // one wave of group CTAs
     const int by_work = max(1, NG / (2 * kWarps));                 // >= 2 groups per warp
     splits_g = max(1, min(min(want, by_work), a.max_splits - kMaxResidualChunks));

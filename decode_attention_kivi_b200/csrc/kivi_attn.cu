@@ -42,6 +42,10 @@ namespace {
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 constexpr int kStages = 4;
+// Row stride (fp16 entries) of a warp's p tile [8 heads][64 tokens]: 64 plus 8 of
+// padding, so that the eight rows a P.V operand load touches fall in distinct
+// banks (a 64-entry row is 128 bytes: every row would start in bank 0).
+constexpr int kPRow = 2 * 32 + 8;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr long long kWaitBudgetCycles = 4000000000LL;  // about 2 s at 1.9 GHz
 constexpr uint32_t kStatusWaitTimeout = 1u;
@@ -215,7 +219,7 @@ struct Plan {
   static constexpr RecordGeom geo{D, BITS};
   static constexpr int kRec = (int)geo.bytes();             // bytes, multiple of 128
   static constexpr int kStageBytes = kWarps * kStages * kRec;
-  static constexpr int kPBytes = kWarps * 8 * 2 * kGroup * 2;  // per warp p[8 heads][64] fp16
+  static constexpr int kPBytes = kWarps * 8 * kPRow * 2;  // per warp p[8 heads][kPRow] fp16
   static constexpr int kQBytes = HPK * D * 4;               // q (fp32) of this kv head
   static constexpr int kMergeBytes = kWarps * HPK * D * 4;  // aliases the stages
   static_assert(kMergeBytes <= kStageBytes, "merge area must fit in the stage area");
@@ -301,7 +305,7 @@ decode_kernel(DecodeArgs args, int splits_g, int n_res, int groups_per_cta, floa
     const int g = lane >> 2, tig = lane & 3;
     unsigned char* stage0 = smem + warp * kStages * P::kRec;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P::kOffBar) + warp * kStages;
-    __half* p_s = reinterpret_cast<__half*>(smem + P::kOffP) + warp * 8 * 2 * kGroup;
+    __half* p_s = reinterpret_cast<__half*>(smem + P::kOffP) + warp * 8 * kPRow;
 
     // This warp's groups: first + warp, first + warp + kWarps, ...
     const int first = split * groups_per_cta;
@@ -309,7 +313,7 @@ decode_kernel(DecodeArgs args, int splits_g, int n_res, int groups_per_cta, floa
     const int n_mine = first + warp < last ? (last - first - warp + kWarps - 1) / kWarps : 0;
     const uint8_t* seq_rec = args.records + seq * args.ngcap * (long)P::kRec;
 
-    for (int i = lane; i < 8 * 2 * kGroup / 2; i += 32)
+    for (int i = lane; i < 8 * kPRow / 2; i += 32)
       reinterpret_cast<uint32_t*>(p_s)[i] = 0u;  // heads without a query stay finite
     if (lane == 0) {
       for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
@@ -500,7 +504,7 @@ decode_kernel(DecodeArgs args, int splits_g, int n_res, int groups_per_cta, floa
         alpha[c] = fast_exp2(m_run[c] - m_new);
         m_run[c] = m_new;
         float sum = 0.f;
-        __half* prow = p_s + (4 * c + tig) * 2 * kGroup;
+        __half* prow = p_s + (4 * c + tig) * kPRow;
 #pragma unroll
         for (int grp = 0; grp < 2; ++grp)
 #pragma unroll
@@ -557,7 +561,7 @@ decode_kernel(DecodeArgs args, int splits_g, int n_res, int groups_per_cta, floa
         for (int kk = 0; kk < 2; ++kk)
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf)
-            pb[kk][hf] = *reinterpret_cast<const uint32_t*>(p_s + g * 2 * kGroup + grp * kGroup +
+            pb[kk][hf] = *reinterpret_cast<const uint32_t*>(p_s + g * kPRow + grp * kGroup +
                                                             16 * kk + 8 * hf + 2 * tig);
         // value-min term, deferred: rows g -> block g % kBlocks
         {

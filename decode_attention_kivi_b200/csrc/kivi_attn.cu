@@ -797,23 +797,51 @@ decode_kernel(DecodeArgs args, int splits_g, int n_res, int groups_per_cta, floa
 }
 
 // out[b][h] = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s.
+// Warp 0 reads every split's (m, l) at once (two per lane, splits <= 64) and
+// reduces them with shuffles; then every thread sums its channel over the
+// splits with independent loads.
 template <int D>
 __global__ void __launch_bounds__(D) combine_kernel(DecodeArgs args, int splits) {
+  static_assert(D >= 64, "warp 0 and the split weights need D >= 64 threads");
+  __shared__ float f_s[kMaxSplitsCap];
+  __shared__ float inv_l;
   wait_for_predecessor();  // every split's partial is written
   allow_successor();
   const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
   const long part0 = ((long)b * args.Hq + h) * splits;
-  float M = -INFINITY;
-  for (int s = 0; s < splits; ++s) M = fmaxf(M, args.ws_ml[2 * (part0 + s)]);
-  float L = 0.f, o = 0.f;
-  for (int s = 0; s < splits; ++s) {
-    const float ms = args.ws_ml[2 * (part0 + s)];
-    if (ms == -INFINITY) continue;
-    const float f = exp2f(ms - M);
-    L += f * args.ws_ml[2 * (part0 + s) + 1];
-    o += f * args.ws_acc[(part0 + s) * D + d];
+  if (d < 32) {
+    float m[2], l[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int s = d + 32 * k;
+      m[k] = s < splits ? args.ws_ml[2 * (part0 + s)] : -INFINITY;
+      l[k] = s < splits ? args.ws_ml[2 * (part0 + s) + 1] : 0.f;
+    }
+    float M = fmaxf(m[0], m[1]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float L = 0.f;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const float f = m[k] == -INFINITY ? 0.f : exp2f(m[k] - M);
+      if (d + 32 * k < splits) f_s[d + 32 * k] = f;
+      L += f * l[k];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    if (d == 0) inv_l = 1.f / L;
   }
-  args.out[((long)b * args.Hq + h) * D + d] = o / L;
+  __syncthreads();
+  const float* acc = args.ws_acc + part0 * D + d;
+  float o0 = 0.f, o1 = 0.f;
+  int s = 0;
+#pragma unroll 4
+  for (; s + 1 < splits; s += 2) {
+    o0 = fmaf(f_s[s], acc[(long)s * D], o0);
+    o1 = fmaf(f_s[s + 1], acc[(long)(s + 1) * D], o1);
+  }
+  if (s < splits) o0 = fmaf(f_s[s], acc[(long)s * D], o0);
+  args.out[((long)b * args.Hq + h) * D + d] = (o0 + o1) * inv_l;
 }
 
 template <int D, int BITS, int HPK>

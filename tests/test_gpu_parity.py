@@ -110,6 +110,12 @@ def test_small_shapes(kivi, D, bits, hpk):
                seed=D + bits + hpk, check_each=False)
 
 
+def test_many_splits(kivi):
+    """One sequence and kv head at 8K tokens: 28 group splits plus 5 residual chunks, so the
+    combine merges more than 32 partials (two per lane of its first warp)."""
+    _run_small(kivi, B=1, Hkv=1, Hq=4, D=128, bits=2, S0=8192, steps=1, seed=91)
+
+
 def test_decode_without_prefill(kivi):
     """Append-only growth from an empty layer through the first flush."""
     _run_small(kivi, B=1, Hkv=1, Hq=1, D=128, bits=2, S0=0, steps=165, seed=5, check_each=False)

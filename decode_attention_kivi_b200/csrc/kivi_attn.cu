@@ -228,8 +228,7 @@ struct Plan {
   static constexpr int kOffP = kStageBytes;
   static constexpr int kOffQ = kOffP + kPBytes;
   static constexpr int kOffML = kOffQ + kQBytes;               // wm, wl [kWarps][8] each
-  static constexpr int kOffExp = kOffML + 2 * kWarps * 8 * 4;  // e_h [8] ints
-  static constexpr int kOffBar = kOffExp + 8 * 4;              // [kWarps][kStages] mbarriers
+  static constexpr int kOffBar = kOffML + 2 * kWarps * 8 * 4;  // [kWarps][kStages] mbarriers
   static constexpr int kBytes = kOffBar + kWarps * kStages * 8;
 };
 
@@ -256,7 +255,6 @@ decode_kernel(DecodeArgs args, int splits_g, int n_res, int groups_per_cta, floa
   float* q_s = reinterpret_cast<float*>(smem + P::kOffQ);
   float* wm = reinterpret_cast<float*>(smem + P::kOffML);
   float* wl = wm + kWarps * 8;
-  int* exp_s = reinterpret_cast<int*>(smem + P::kOffExp);
 
   const int n_group_ctas = splits_g * args.Hkv * args.B;
   int split, kvh, b;
@@ -275,76 +273,94 @@ decode_kernel(DecodeArgs args, int splits_g, int n_res, int groups_per_cta, floa
   const long seq = (long)b * args.Hkv + kvh;
   const int NG = num_groups(S);
 
-  wait_for_predecessor();  // q, the records and the rings may come from the previous kernel
-  // q of this kv head's query heads, fp32 in smem; per-head exponent e_h with
-  // max |q_h| * 2^-e_h in [0.5, 1).
-  for (int i = threadIdx.x; i < HPK * D; i += kThreads) {
-    const int hh = i / D, d = i % D;
-    q_s[i] = __bfloat162float(args.q[((long)b * Hq + kvh * HPK + hh) * D + d]);
-  }
-  __syncthreads();
-  if (warp == 0 && split < splits_g) {  // the residual CTAs do not scale q
-    for (int hh = 0; hh < HPK; ++hh) {
-      float mx = 0.f;
-      for (int d = lane; d < D; d += 32) mx = fmaxf(mx, fabsf(q_s[hh * D + d]));
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      if (lane == 0) {
-        int e = 0;
-        if (mx > 0.f) frexpf(mx, &e);
-        exp_s[hh] = e;
-      }
-    }
-  }
-  __syncthreads();
-
+  const bool group_cta = split < splits_g;
+  const int g = lane >> 2, tig = lane & 3;
   float* merge_acc = reinterpret_cast<float*>(smem);  // [kWarps][HPK][D], used after the loop
-
-  if (split < splits_g) {
-    // ===================== group CTA: tensor-core path =====================
-    const int g = lane >> 2, tig = lane & 3;
-    unsigned char* stage0 = smem + warp * kStages * P::kRec;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P::kOffBar) + warp * kStages;
-    __half* p_s = reinterpret_cast<__half*>(smem + P::kOffP) + warp * 8 * kPRow;
-
-    // This warp's groups: first + warp, first + warp + kWarps, ...
-    const int first = split * groups_per_cta;
-    const int last = min(NG, first + groups_per_cta);
-    const int n_mine = first + warp < last ? (last - first - warp + kWarps - 1) / kWarps : 0;
-    const uint8_t* seq_rec = args.records + seq * args.ngcap * (long)P::kRec;
-
+  // Group-CTA geometry: this warp's groups are first + warp, first + warp + kWarps, ...
+  unsigned char* stage0 = smem + warp * kStages * P::kRec;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P::kOffBar) + warp * kStages;
+  __half* p_s = reinterpret_cast<__half*>(smem + P::kOffP) + warp * 8 * kPRow;
+  const int first = split * groups_per_cta;
+  const int last = min(NG, first + groups_per_cta);
+  const int n_mine =
+      group_cta && first + warp < last ? (last - first - warp + kWarps - 1) / kWarps : 0;
+  const uint8_t* seq_rec = args.records + seq * args.ngcap * (long)P::kRec;
+  if (group_cta) {
     for (int i = lane; i < 8 * kPRow / 2; i += 32)
       reinterpret_cast<uint32_t*>(p_s)[i] = 0u;  // heads without a query stay finite
     if (lane == 0) {
       for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
       fence_mbar_init();
     }
-    __syncwarp();
-    if (lane == 0) {
-      for (int i = 0; i < kStages && i < n_mine; ++i) {
-        mbar_expect_tx(&bars[i], P::kRec);
-        bulk_load(stage0 + i * P::kRec, seq_rec + (long)(first + warp + i * kWarps) * P::kRec,
-                  P::kRec, &bars[i]);
-      }
-    }
+  }
 
+  wait_for_predecessor();  // q, the records and the rings may come from the previous kernel
+  // q of this kv head's query heads (16-byte pieces): the loads go out before
+  // the record stream so that they do not queue behind it
+  constexpr int kQPieces = HPK * D / 8;
+  static_assert(kQPieces <= kThreads, "one 16-byte piece of q per thread");
+  uint4 qv = make_uint4(0u, 0u, 0u, 0u);
+  if (threadIdx.x < kQPieces)  // the heads of kv head kvh are contiguous
+    qv = reinterpret_cast<const uint4*>(args.q + ((long)b * Hq + kvh * HPK) * D)[threadIdx.x];
+  if (group_cta && lane == 0) {
+    for (int i = 0; i < kStages && i < n_mine; ++i) {
+      mbar_expect_tx(&bars[i], P::kRec);
+      bulk_load(stage0 + i * P::kRec, seq_rec + (long)(first + warp + i * kWarps) * P::kRec,
+                P::kRec, &bars[i]);
+    }
+  }
+  if (threadIdx.x < kQPieces) {  // q as fp32 in smem
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&qv);
+    float4* dst = reinterpret_cast<float4*>(q_s + threadIdx.x * 8);
+    const float2 f0 = __bfloat1622float2(h2[0]), f1 = __bfloat1622float2(h2[1]);
+    const float2 f2 = __bfloat1622float2(h2[2]), f3 = __bfloat1622float2(h2[3]);
+    dst[0] = make_float4(f0.x, f0.y, f1.x, f1.y);
+    dst[1] = make_float4(f2.x, f2.y, f3.x, f3.y);
+  }
+  __syncthreads();
+
+  if (group_cta) {
+    // ===================== group CTA: tensor-core path =====================
     CodeConsts<BITS> kc;
     kc.init();
 
     // Score B operand: column n = g is head 4c + g/2 of chunk c, hi part for even
     // g and lo part for odd g.  qq = q''[head][channels c0..c0+3] per k-step,
     // c0 = tig*D/4 + 4s.  negm = -1 (odd g) or 0 (even g) in fp16x2.
+    // Per-head exponent e_h with max |q_h| 2^-e_h in [0.5, 1), computed by every
+    // warp: lanes [h L, (h+1) L) take head h (L = 32 / HPK lanes, D / L values each).
+    int ex[HPK];
+    {
+      constexpr int kLanesPerHead = 32 / HPK;
+      constexpr int kPerLane = D / kLanesPerHead;
+      const float* qh = q_s + (lane / kLanesPerHead) * D + (lane % kLanesPerHead) * kPerLane;
+      float mx = 0.f;
+#pragma unroll
+      for (int i = 0; i < kPerLane; ++i) mx = fmaxf(mx, fabsf(qh[i]));
+#pragma unroll
+      for (int o = 1; o < kLanesPerHead; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      int e = 0;
+      if (mx > 0.f) frexpf(mx, &e);
+#pragma unroll
+      for (int hh = 0; hh < HPK; ++hh) ex[hh] = __shfl_sync(0xffffffffu, e, hh * kLanesPerHead);
+    }
     uint32_t qq[kChunks][kKSteps][2];
     const uint32_t negm = (g & 1) ? 0xBC00BC00u : 0u;
     float ch[kChunks];  // log2 score scale of head 4c + tig
 #pragma unroll
     for (int c = 0; c < kChunks; ++c) {
       const int hs = 4 * c + g / 2;
+      int es = 0, et = 0;
+#pragma unroll
+      for (int hh = 0; hh < HPK; ++hh) {
+        es = hh == hs ? ex[hh] : es;
+        et = hh == 4 * c + tig ? ex[hh] : et;
+      }
 #pragma unroll
       for (int s = 0; s < kKSteps; ++s) {
         const int c0 = tig * (D / 4) + 4 * s;
         if (hs < HPK) {
-          const float sc = ldexpf(1.f, -exp_s[hs]);
+          const float sc = ldexpf(1.f, -es);
           const float* qr = q_s + hs * D + c0;
           qq[c][s][0] = pack_half2(qr[0] * sc, qr[1] * sc);
           qq[c][s][1] = pack_half2(qr[2] * sc, qr[3] * sc);
@@ -353,7 +369,7 @@ decode_kernel(DecodeArgs args, int splits_g, int n_res, int groups_per_cta, floa
         }
       }
       const int hh = 4 * c + tig;
-      ch[c] = hh < HPK ? ldexpf(qscale, exp_s[hh]) : 1.f;  // > 0 keeps -inf scores at p = 0
+      ch[c] = hh < HPK ? ldexpf(qscale, et) : 1.f;  // > 0 keeps -inf scores at p = 0
     }
 
     float acc[kMTiles][4];

@@ -8,7 +8,8 @@
 // R tokens stay full precision).  Grouped history and residual share one
 // online softmax.
 //
-// Group CTAs (blockIdx.x < splits_g): each warp streams whole 32-token group
+// Group CTAs (split < splits_g of each sequence and kv head; one wave of 4 CTAs
+// per SM): each warp streams whole 32-token group
 // records (one contiguous block each) into its own shared-memory ring with
 // cp.async.bulk on mbarriers, and does both contractions on the tensor cores
 // (mma.sync m16n8k16, fp16 operands, fp32 accumulation):
@@ -18,14 +19,15 @@
 //           the code operand) so the scores keep about 22 significant bits
 //   P.V     C[chan][head] += sum_t code[t][chan] * (p[head][t] * vscale[t][j])
 //                          + sum_t vmin[t][j] * p[head][t]
-// The codes become exact fp16 small integers with one mask-and-or and one fma
-// per pair (the packing puts adjacent codes in the two halves of a word); the
+// The codes become exact fp16 small integers with one three-input logic op and
+// one add per pair (the packing puts adjacent codes in the two halves of a word); the
 // scale and the min fold into the other operand, so nothing is dequantized
 // element by element.  The min terms are MMAs whose A rows all repeat the min
 // vector.  q'' = q * 2^-e_h (exact) keeps |q''| < 1 so q'' * kscale stays in
 // fp16 range; scores are rescaled by 2^e_h * sm_scale * log2(e) in fp32.
 //
-// Residual CTA (blockIdx.x == splits_g): the bf16 ring tokens on CUDA cores.
+// Residual-chunk CTAs (after the group CTAs in the grid; they fill the SMs the
+// group CTAs leave free): 32 bf16 ring tokens each, on CUDA cores.
 // Every CTA writes one (m, l, acc) partial per query head; combine_kernel
 // merges the partials.  Every wait on an mbarrier is bounded; a wait that runs
 // out sets the device status word and the CTA stops issuing work.
@@ -240,7 +242,7 @@ template <int D, int BITS, int HPK>
 __global__ void __launch_bounds__(kThreads, HPK <= 4 ? 4 : 2)
 decode_kernel(DecodeArgs args, int splits_g, int n_res, int groups_per_cta, float qscale) {
   // Linear grid: B*Hkv*splits_g group CTAs (split fastest), then B*Hkv*n_res
-  // residual-chunk CTAs, so the short residual CTAs run last and fill the tail.
+  // residual-chunk CTAs, which take the slots the group CTAs leave free.
   using P = Plan<D, BITS, HPK>;
   using CW = CodeWord<BITS>;
   constexpr RecordGeom geo = P::geo;

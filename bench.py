@@ -21,6 +21,7 @@ import re
 import statistics
 import subprocess
 import sys
+import threading
 import time
 
 import torch
@@ -140,8 +141,17 @@ class ClockSampler:
     def __init__(self, device_index: int):
         self.device_index = device_index
         self.proc = None
+        self.lines = []
+        self.reader = None
+        self.t_start = 0.0
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.monotonic(), line))
 
     def start(self):
+        """Starts nvidia-smi and returns once it has printed its first sample, so that
+        the (short) timed region that follows is sampled from its start."""
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.device_index}", f"--query-gpu={self.FIELDS}",
@@ -149,16 +159,26 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+            return
+        self.reader = threading.Thread(target=self._read, daemon=True)
+        self.reader.start()
+        deadline = time.monotonic() + 5.0
+        while not self.lines and self.proc.poll() is None and time.monotonic() < deadline:
+            time.sleep(0.005)
+        self.t_start = time.monotonic()
 
     def stop(self) -> dict:
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
         try:
-            out, _ = self.proc.communicate(timeout=5)
+            self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-            out, _ = self.proc.communicate()
+            self.proc.wait()
+        self.reader.join(timeout=5)
+        timed = [line for t, line in self.lines if t >= self.t_start]
+        out = "".join(timed if timed else [line for _, line in self.lines])
         sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in out.strip().splitlines():

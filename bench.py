@@ -83,12 +83,51 @@ def weak_scaling_tokens_per_s(world: int, batch: int, steps: int, ms: float) -> 
     return world * batch * steps / (ms * 1e-3)
 
 
-def workload_config(w: synth.Workload, s_first: int, s_last: int, l2_note: str) -> dict:
+def flush_steps(context: int, first: int, count: int) -> list:
+    """Indices i in [first, first + count) of the decode steps (step i appends token
+    context + i) whose append flushes 32 residual tokens into a new group: the
+    residual would reach R + G = 160 tokens."""
+    out = []
+    for i in range(first, first + count):
+        S = context + i
+        ng = 0 if S < 128 else (S - 128) // 32
+        if S + 1 - 32 * ng == 160:
+            out.append(i)
+    return out
+
+
+def timed_window(context: int, warmup: int, steps: int) -> int:
+    """Untimed steps before the timed window: at least `warmup`, chosen so that the
+    window of `steps` steps holds a residual flush as near its middle as possible (a
+    flush comes every 32 steps)."""
+    best, best_d = warmup, None
+    for pre in range(warmup, warmup + 32):
+        fl = flush_steps(context, pre, steps)
+        if not fl:
+            continue
+        d = min(abs(f - (pre + steps // 2)) for f in fl)
+        if best_d is None or d < best_d:
+            best, best_d = pre, d
+    return best
+
+
+def workload_config(w: synth.Workload, warmup: int, steps: int) -> dict:
+    """The workload and the timed window, identical in both arms."""
+    pre = timed_window(w.context, warmup, steps)
     return {"workload": w.name, "batch_per_gpu": w.batch, "layers": w.num_layers,
             "kv_heads": w.num_kv_heads, "q_heads": w.num_q_heads, "head_dim": w.head_dim,
             "bits": w.bits, "group_size": 32, "residual": 128, "prefill_context": w.context,
-            "context_at_timed_steps": [s_first, s_last], "l2": l2_note,
+            "untimed_steps_before_window": pre,
+            "context_at_timed_steps": [w.context + pre + 1, w.context + pre + steps],
+            "residual_flushes_in_window": len(flush_steps(w.context, pre, steps)),
             "step": "per layer: kivi_append_token (flush when due) + kivi_decode_attention"}
+
+
+def percentiles(xs) -> dict:
+    ys = sorted(xs)
+    pick = lambda f: ys[min(len(ys) - 1, max(0, int(round(f * (len(ys) - 1)))))]
+    return {"median": statistics.median(ys), "p10": pick(0.10), "p90": pick(0.90),
+            "mean": sum(ys) / len(ys), "n": len(ys)}
 
 
 def hbm_peak():
@@ -214,14 +253,18 @@ def build_cache(K, w: synth.Workload, max_tokens: int, device):
     return cache
 
 
-def run_gpu(args, w: synth.Workload, rank: int, world: int):
+L2_FLUSH_BYTES = 512 << 20  # more than 4x B200's 126 MB L2
+
+
+def run_gpu(args, w: synth.Workload, cfg: dict, rank: int, world: int):
     import decode_attention_kivi_b200 as K
     from decode_attention_kivi_b200._native import lib
 
     device = torch.device("cuda", torch.cuda.current_device())
-    steps, warmup = args.steps, args.warmup
-    total_steps = warmup + steps + (0 if args.no_e2e else warmup + steps)
-    cache = build_cache(K, w, w.context + total_steps + 1, device)
+    steps = args.steps
+    pre = cfg["untimed_steps_before_window"]
+    e2e_steps = 0 if args.no_e2e else args.warmup + steps
+    cache = build_cache(K, w, w.context + pre + steps + e2e_steps + 1, device)
     L = lib()
     stream = torch.cuda.current_stream()
     sptr = stream.cuda_stream
@@ -235,6 +278,11 @@ def run_gpu(args, w: synth.Workload, rank: int, world: int):
     kp = [a.data_ptr() for a, _ in kv]
     vp = [b.data_ptr() for _, b in kv]
     op = [out[l].data_ptr() for l in range(w.num_layers)]
+    # One step reads every layer's cache; when that is not far above L2, a buffer
+    # larger than L2 is written between timed steps (outside their events).
+    step_bytes = w.num_layers * attention_bytes(w, w.context + pre)
+    flush_l2 = step_bytes < 4 * 126e6
+    scratch = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device) if flush_l2 else None
 
     def check(rc, what):
         if rc != 0:
@@ -249,28 +297,29 @@ def run_gpu(args, w: synth.Workload, rank: int, world: int):
             if ev is not None:
                 ev[l][1].record(stream)
 
-    for _ in range(warmup):
+    for _ in range(pre):
         step()
     torch.cuda.synchronize()
     s_first = cache.length(0)[0] + 1
-    # per-launch events of the attention calls over the timed region
-    evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
-            for _ in range(w.num_layers)] for _ in range(steps)]
-    bytes_timed = 0
-    for i in range(steps):
-        bytes_timed += w.num_layers * attention_bytes(w, s_first + i)
+    new = lambda: torch.cuda.Event(enable_timing=True)
+    evs = [[[new(), new()] for _ in range(w.num_layers)] for _ in range(steps)]
+    st_ev = [[new(), new()] for _ in range(steps)]
+    bytes_timed = sum(w.num_layers * attention_bytes(w, s_first + i) for i in range(steps))
     sampler = ClockSampler(device.index if device.index is not None else 0)
     sampler.start()
     time.sleep(0.05)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
+    t0, t1 = new(), new()
     torch.cuda.nvtx.range_push("kivi_timed_steps")  # lets ncu --nvtx-include select these launches
     t0.record(stream)
     for i in range(steps):
+        if scratch is not None:
+            scratch.zero_()
+        st_ev[i][0].record(stream)
         step(evs[i])
+        st_ev[i][1].record(stream)
     t1.record(stream)
     torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
@@ -278,12 +327,13 @@ def run_gpu(args, w: synth.Workload, rank: int, world: int):
         torch.distributed.barrier()
     clocks = sampler.stop()
     s_last = cache.length(0)[0]
-    ms = t0.elapsed_time(t1)
-    attn_ms = sum(e[0].elapsed_time(e[1]) for st in evs for e in st)
-    n_attn = steps * w.num_layers
+    ms = (sum(a.elapsed_time(b) for a, b in st_ev) if flush_l2 else t0.elapsed_time(t1))
+    call_us = [1e3 * e[0].elapsed_time(e[1]) for stp in evs for e in stp]
+    attn_ms = 1e-3 * sum(call_us)
     # device status after the timed region (bounded waits report here)
     if cache.check_device_status() != 0:
         raise RuntimeError("a kernel reported a failure in the device status word")
+    del scratch
 
     e2e = None
     if not args.no_e2e:
@@ -294,13 +344,16 @@ def run_gpu(args, w: synth.Workload, rank: int, world: int):
         if e2e is not None:
             e2e["_ms"] = max_over_ranks([e2e["_ms"]], device)[0]
     cache.close()
-    return dict(ms=ms, attn_ms=attn_ms, n_attn=n_attn, bytes_timed=bytes_timed,
-                s_first=s_first, s_last=s_last, clocks=clocks, e2e=e2e)
+    return dict(ms=ms, attn_ms=attn_ms, call_us=call_us, bytes_timed=bytes_timed,
+                s_first=s_first, s_last=s_last, clocks=clocks, e2e=e2e, flush_l2=flush_l2,
+                step_bytes=step_bytes)
 
 
 def run_e2e(args, w, cache, L, h, sptr, device, world):
     """Same steps through the C ABI with the step's inputs copied from pinned host
-    memory and the step's outputs read back, copies inside the timed region."""
+    memory and the step's outputs read back, copies inside the timed region.  The
+    copies run on their own stream, ordered by events: layer l's inputs arrive
+    while earlier layers compute, and layer l's output leaves while later layers do."""
     nl = w.num_layers
     hq = [synth.query(w, l, 1).pin_memory() for l in range(nl)]
     hk = [synth.step_kv(w, l, 1)[0].pin_memory() for l in range(nl)]
@@ -312,30 +365,52 @@ def run_e2e(args, w, cache, L, h, sptr, device, world):
     dout = torch.empty(hout.shape, dtype=torch.float32, device=device)
     h2d = sum(t.numel() * t.element_size() for t in hq + hk + hv)
     d2h = hout.numel() * hout.element_size()
+    comp = torch.cuda.current_stream()
+    copy = torch.cuda.Stream(device=device)
+    inputs_in = [torch.cuda.Event() for _ in range(nl)]
+    inputs_used = [torch.cuda.Event() for _ in range(nl)]
+    out_ready = [torch.cuda.Event() for _ in range(nl)]
+    out_read = [torch.cuda.Event() for _ in range(nl)]
+    first = [True]
 
     def step():
         for l in range(nl):
-            dq[l].copy_(hq[l], non_blocking=True)
-            dk[l].copy_(hk[l], non_blocking=True)
-            dv[l].copy_(hv[l], non_blocking=True)
+            with torch.cuda.stream(copy):
+                if not first[0]:
+                    copy.wait_event(inputs_used[l])  # the previous step's layer l is done with them
+                dq[l].copy_(hq[l], non_blocking=True)
+                dk[l].copy_(hk[l], non_blocking=True)
+                dv[l].copy_(hv[l], non_blocking=True)
+                inputs_in[l].record(copy)
+        for l in range(nl):
+            comp.wait_event(inputs_in[l])
+            if not first[0]:
+                comp.wait_event(out_read[l])  # the previous step's output of layer l has left
             rc = L.kivi_append_token(h, l, dk[l].data_ptr(), dv[l].data_ptr(), sptr)
             rc |= L.kivi_decode_attention(h, l, dq[l].data_ptr(), dout[l].data_ptr(), 0.0, sptr)
             if rc:
                 raise RuntimeError("kivi call failed in the e2e loop")
-        hout.copy_(dout, non_blocking=True)
+            inputs_used[l].record(comp)
+            out_ready[l].record(comp)
+            with torch.cuda.stream(copy):
+                copy.wait_event(out_ready[l])
+                hout[l].copy_(dout[l], non_blocking=True)
+                out_read[l].record(copy)
+        first[0] = False
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
-    stream = torch.cuda.current_stream()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
+    t0.record(comp)
+    copy.wait_stream(comp)  # no copy of the timed steps starts before t0
     for _ in range(args.steps):
         step()
-    t1.record(stream)
+    comp.wait_stream(copy)  # the last step's outputs are on the host
+    t1.record(comp)
     torch.cuda.synchronize()
     assert torch.isfinite(hout).all()
     return {"_ms": t0.elapsed_time(t1), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
@@ -345,15 +420,24 @@ def run_e2e(args, w, cache, L, h, sptr, device, world):
 # The oracle on the host cores (CPU baseline and the reference arm)
 # ---------------------------------------------------------------------------
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 class OracleSample:
     """One layer of the workload in the oracle, at the prefill context."""
 
     def __init__(self, w: synth.Workload):
-        import numpy as np
-
         import oracle as O
 
-        self.np, self.O, self.w = np, O, w
+        self.O, self.w = O, w
         k, v = synth.prefill_kv(w, 0)
         self.cache = O.OracleCache(w.batch, w.num_kv_heads, w.head_dim, w.bits,
                                    w.context + 4096)
@@ -362,57 +446,153 @@ class OracleSample:
         self.kn, self.vn = synth.bf16_bits(kn), synth.bf16_bits(vn)
         self.q = synth.bf16_bits(synth.query(w, 0, 0))
         self.rows = [(b, h) for b in range(w.batch) for h in range(w.num_q_heads)]
+        self.next = 0
 
-    def step_seconds(self, n_rows: int, start: int = 0) -> float:
-        """Projected seconds of one full decode step from timing n_rows attention
-        rows (of B*Hq) and one append of one layer, scaled to all rows and layers."""
-        w = self.w
+    def time_rows(self, n_rows: int):
+        """Seconds for one append of the layer and n_rows attention rows."""
         t0 = time.perf_counter()
         self.cache.append(self.kn, self.vn)
         t_append = time.perf_counter() - t0
         t0 = time.perf_counter()
-        for i in range(n_rows):
-            b, hh = self.rows[(start + i) % len(self.rows)]
-            self.cache.attend(b, hh, self.q[b, hh], w.num_q_heads)
-        t_rows = time.perf_counter() - t0
-        per_layer = t_append + t_rows * len(self.rows) / n_rows
-        return per_layer * w.num_layers
+        for _ in range(n_rows):
+            b, hh = self.rows[self.next % len(self.rows)]
+            self.next += 1
+            self.cache.attend(b, hh, self.q[b, hh], self.w.num_q_heads)
+        return t_append, time.perf_counter() - t0
 
 
-def cpu_baseline(w: synth.Workload, budget_s: float = 12.0) -> dict:
-    s = OracleSample(w)
+_WORKER_SAMPLE = None
+
+
+def _oracle_worker_init(name, batch, layers, worker_index):
+    global _WORKER_SAMPLE
+    w = dataclasses.replace(synth.WORKLOADS[name], batch=batch, num_layers=layers)
+    _WORKER_SAMPLE = OracleSample(w)
+    _WORKER_SAMPLE.next = worker_index * 7
+
+
+def _oracle_worker_rows(n_rows):
+    return _WORKER_SAMPLE.time_rows(n_rows)
+
+
+class OracleTimer:
+    """The plain C oracle on the host: single-threaded in this process, and one
+    worker process per core (spawned, no CUDA) timing rows side by side."""
+
+    def __init__(self, w: synth.Workload, workers: int):
+        import multiprocessing as mp
+
+        self.w = w
+        self.rows_per_step = w.num_layers * w.batch * w.num_q_heads
+        self.workers = workers
+        self.pool = None
+        if workers > 1:
+            ctx = mp.get_context("spawn")
+            # one pool of `workers` processes, each holding its own oracle copy
+            self.pool = ctx.Pool(workers, initializer=_oracle_worker_init,
+                                 initargs=(w.name, w.batch, w.num_layers, 0))
+            self.pool.map(_oracle_worker_rows, [1] * workers)  # builds the copies
+
+    def all_cores(self, rows_each: int) -> dict:
+        """Rows/s with every worker timing rows_each rows at once (wall clock)."""
+        t0 = time.perf_counter()
+        res = self.pool.map(_oracle_worker_rows, [rows_each] * self.workers, chunksize=1)
+        wall = time.perf_counter() - t0
+        rows = rows_each * self.workers
+        return {"rows": rows, "seconds": wall, "rows_per_s": rows / wall,
+                "append_s": max(a for a, _ in res)}
+
+    def close(self):
+        if self.pool is not None:
+            self.pool.close()
+            self.pool.join()
+
+
+def _projection(w, rows_per_s):
+    rows_per_step = w.num_layers * w.batch * w.num_q_heads
+    step_s = rows_per_step / rows_per_s
+    return step_s, w.batch / step_s
+
+
+def cpu_baseline(w: synth.Workload, budget_s: float = 20.0) -> dict:
+    """The oracle as it stands, on a bounded sample of the workload: attention rows
+    (sequence, query head) of one layer at the prefill context, timed and projected
+    to a full decode step (every row of every layer)."""
+    workers = os.cpu_count() or 1
+    single = OracleSample(w)
     t_start = time.perf_counter()
-    rows_done, proj = 0, []
-    while time.perf_counter() - t_start < budget_s and rows_done < len(s.rows):
-        n = 8
-        proj.append(s.step_seconds(n, rows_done))
-        rows_done += n
-    step_s = statistics.median(proj)
-    return {"value": w.batch / step_s, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": (f"{rows_done} of {len(s.rows)} (sequence, query head) attention rows of "
-                       f"layer 0 at S={w.context}+ plus one append per 8 rows, in "
-                       f"{len(proj)} batches; scaled to all rows and {w.num_layers} layers; "
-                       "single-threaded plain C oracle")}
+    rows1, sec1 = 0, 0.0
+    while time.perf_counter() - t_start < 0.3 * budget_s:
+        _, t = single.time_rows(4)
+        rows1 += 4
+        sec1 += t
+    timer = OracleTimer(w, workers)
+    try:
+        done, sec, rows = 0, 0.0, 0
+        t_start = time.perf_counter()
+        while time.perf_counter() - t_start < 0.5 * budget_s:
+            r = timer.all_cores(2)
+            rows += r["rows"]
+            sec += r["seconds"]
+    finally:
+        timer.close()
+    rate = rows / sec if workers > 1 else rows1 / sec1
+    step_s, value = _projection(w, rate)
+    step1_s, value1 = _projection(w, rows1 / sec1)
+    return {"value": value, "unit": "tokens/s", "cores": workers, "threads": workers,
+            "cpu_model": cpu_model(), "kind": "oracle", "projected": True,
+            "rows_measured": rows, "rows_per_s": rate,
+            "rows_per_step": timer.rows_per_step,
+            "scale_factor": timer.rows_per_step / max(rows, 1),
+            "single_thread": {"value": value1, "rows_measured": rows1,
+                              "rows_per_s": rows1 / sec1},
+            "sample": (f"{rows} attention rows (sequence, query head) of layer 0 at S="
+                       f"{w.context}+, {workers} worker processes side by side (one per "
+                       f"core, {cpu_model()}); a full decode step is "
+                       f"{timer.rows_per_step} rows ({w.num_layers} layers), so the "
+                       f"figure is projected from the measured rows/s; plain C oracle, "
+                       "fp64 accumulation")}
 
 
-def run_reference(args, w: synth.Workload):
-    s = OracleSample(w)
-    n = 8
-    for i in range(args.warmup):
-        s.step_seconds(n, i * n)
-    total = 0.0
-    for i in range(args.steps):
-        total += s.step_seconds(n, (args.warmup + i) * n)
-    value = w.batch * args.steps / total
-    sample = (f"each step: {n} of {w.batch * w.num_q_heads} (sequence, query head) attention "
-              f"rows of one layer plus one append, timed and scaled to all rows and "
-              f"{w.num_layers} layers; single-threaded plain C oracle")
+def run_reference(args, w: synth.Workload, cfg: dict):
+    workers = os.cpu_count() or 1
+    timer = OracleTimer(w, workers) if workers > 1 else None
+    single = OracleSample(w) if workers == 1 else None
+    rows_each = 2
+    try:
+        def one_step():
+            if timer is not None:
+                r = timer.all_cores(rows_each)
+                return r["rows"], r["seconds"]
+            _, t = single.time_rows(rows_each)
+            return rows_each, t
+        for _ in range(args.warmup):
+            one_step()
+        rows, sec = 0, 0.0
+        for _ in range(args.steps):
+            r, t = one_step()
+            rows += r
+            sec += t
+    finally:
+        if timer is not None:
+            timer.close()
+    rate = rows / sec
+    step_s, value = _projection(w, rate)
+    rows_per_step = w.num_layers * w.batch * w.num_q_heads
+    sample = (f"each step: {rows_each * workers} of the {rows_per_step} attention rows "
+              f"(sequence, query head) of a decode step, {workers} worker processes side by "
+              f"side (one per core, {cpu_model()}), timed and projected to the full step; "
+              "plain C oracle, fp64 accumulation")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+            "ms_per_step": 1e3 * step_s, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": workload_config(w, w.context + 1, w.context + args.steps, "n/a (host)"),
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "config": cfg, "projected": True,
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": workers,
+                             "threads": workers, "cpu_model": cpu_model(), "kind": "oracle",
+                             "projected": True, "rows_measured": rows, "rows_per_s": rate,
+                             "rows_per_step": rows_per_step,
+                             "scale_factor": rows_per_step * args.steps / rows,
                              "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -430,9 +610,10 @@ def main():
         w = w.with_batch(args.batch)
     if args.layers:
         w = dataclasses.replace(w, num_layers=args.layers)
+    cfg = workload_config(w, args.warmup, args.steps)
     if args.impl == "reference":
         if rank == 0:
-            run_reference(args, w)
+            run_reference(args, w, cfg)
         return
     if world > 1:
         import datetime
@@ -440,27 +621,34 @@ def main():
         local = int(os.environ.get("LOCAL_RANK", "0"))
         torch.cuda.set_device(local)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    res = run_gpu(args, w, rank, world)
+    res = run_gpu(args, w, cfg, rank, world)
     if rank == 0:
         peak, peak_kind = hbm_peak()
+        n_calls = len(res["call_us"])
+        per_launch = res["bytes_timed"] / n_calls
         gbs = res["bytes_timed"] / (res["attn_ms"] * 1e-3) / 1e9
-        per_launch = res["bytes_timed"] / res["n_attn"]
         value = weak_scaling_tokens_per_s(world, w.batch, args.steps, res["ms"])
+        pct = percentiles(res["call_us"])
+        l2 = (f"L2 flushed between timed steps ({L2_FLUSH_BYTES >> 20} MB written, outside "
+              "the step events)" if res["flush_l2"] else
+              f"inputs larger than L2: one step reads every layer's cache "
+              f"({w.num_layers} x ~{per_launch / 1e6:.0f} MB)")
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms"] / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f16 tensor-core operands (codes, q*scale and p*scale as hi+lo pairs; "
+                     "bf16 residual), f32 accumulation",
             "data": "synthetic (seeded; shapes and key-outlier structure of the pages' models)",
-            "config": workload_config(w, res["s_first"], res["s_last"],
-                                      "inputs larger than L2: one step reads every layer's "
-                                      f"cache ({w.num_layers} x ~{per_launch / 1e6:.0f} MB)"),
+            "config": cfg, "l2": l2,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
                          "frac": gbs / peak, "peak_kind": peak_kind,
                          "traffic": recorded_traffic(w),
                          "algorithmic_bytes_per_launch": per_launch,
-                         "kernel": "kivi_decode_attention (split kernel + combine)",
-                         "avg_launch_us": 1e3 * res["attn_ms"] / res["n_attn"]},
-            "gpu_launches": 3 * w.num_layers * args.steps,
+                         "kernel": "decode_kernel (one launch per kivi_decode_attention call)",
+                         "avg_launch_us": pct["mean"],
+                         "launch_us": {k: pct[k] for k in ("median", "p10", "p90", "n")}},
+            "gpu_launches": 2 * w.num_layers * args.steps,
             "clocks": res["clocks"],
         }
         if res["e2e"] is not None:

@@ -21,7 +21,7 @@ __all__ = [
     "kivi_required_bytes", "kivi_cache_create", "kivi_cache_destroy", "kivi_cache_length",
     "kivi_cache_reset", "kivi_quantize_prefill", "kivi_append_token", "kivi_decode_attention",
     "kivi_check_device_status", "kivi_cache_bytes", "kivi_status_string",
-    "kivi_decode_attention_static_scratch",
+    "kivi_decode_attention_static_scratch", "kivi_static_scratch_status",
 ]
 
 GROUP_SIZE = 32
@@ -126,6 +126,16 @@ def kivi_decode_attention_static_scratch(cfg: KiviConfig, records: int, resid_k:
         _ptr(out, torch.float32, "out"), float(sm_scale), _stream(stream)),
         "kivi_decode_attention_static_scratch")
     return out
+
+
+def kivi_static_scratch_status(stream=None) -> int:
+    """Reads and clears the status word of the static-scratch decode call on the
+    current device (0 = no kernel recorded a failure)."""
+    code = ctypes.c_uint32()
+    rc = lib().kivi_static_scratch_status(_stream(stream), ctypes.byref(code))
+    if rc not in (0, 7):
+        check(rc, "kivi_static_scratch_status")
+    return code.value
 
 
 def kivi_check_device_status(handle: int, stream=None) -> int:

@@ -63,6 +63,7 @@ def lib() -> ctypes.CDLL:
         "kivi_status_string": (ctypes.c_char_p, [st]),
         "kivi_decode_attention_static_scratch": (st, [ctypes.POINTER(KiviConfig), P, P, P, I32,
                                                       I32, P, P, F32, P]),
+        "kivi_static_scratch_status": (st, [P, ctypes.POINTER(ctypes.c_uint32)]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)

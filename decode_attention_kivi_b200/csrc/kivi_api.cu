@@ -12,6 +12,7 @@
 
 #include "../../include/kivi.h"
 #include "kivi_kernels.h"
+#include "kivi_launch.cuh"
 #include "kivi_layout.cuh"
 
 struct kivi_cache {
@@ -20,7 +21,6 @@ struct kivi_cache {
   std::vector<int32_t> S;  // token count per layer
   int ngcap;
   long rec_bytes;
-  int max_splits;
   int num_sms;
   int device;
 };
@@ -56,11 +56,27 @@ kivi_sizes sizes_of(const kivi_config* c) {
   s.records_bytes = seqs * ngcap * (size_t)record_bytes(c);
   s.resid_k_bytes = seqs * kRingSlots * (size_t)c->head_dim * 2;
   s.resid_v_bytes = s.resid_k_bytes;
-  const size_t parts = (size_t)c->batch * c->num_q_heads *
-                       kivi::max_splits(c->batch, c->num_kv_heads);
-  s.workspace_bytes = kivi::kWsHeader + parts * 2 * sizeof(float) +
-                      parts * (size_t)c->head_dim * sizeof(float);
+  s.workspace_bytes = (size_t)kivi::decode_workspace_bytes(
+      c->head_dim, c->bits, c->num_q_heads / c->num_kv_heads,
+      (long)c->batch * c->num_kv_heads);
   return s;
+}
+
+long partial_bytes(const kivi_config* c) {
+  return 2L * (c->num_q_heads / c->num_kv_heads) * (c->head_dim + 2) * (long)sizeof(float);
+}
+
+// Points the decode arguments at a workspace of `bytes` bytes: status header,
+// tickets, then as many CTAs' partials as fit.
+void bind_workspace(kivi::DecodeArgs& a, const kivi_config* c, void* ws, size_t bytes) {
+  const long pairs = (long)c->batch * c->num_kv_heads;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  const long fixed = kivi::kWsHeader + kivi::ws_tickets_bytes(pairs);
+  a.status = reinterpret_cast<uint32_t*>(base);
+  a.tickets = reinterpret_cast<int*>(base + kivi::kWsHeader);
+  a.partials = reinterpret_cast<float*>(base + fixed);
+  const long room = (long)bytes - fixed;
+  a.max_ctas = room > 0 ? (int)(room / partial_bytes(c)) : 0;
 }
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
@@ -121,7 +137,10 @@ kivi_status kivi_cache_create(const kivi_config* cfg, const kivi_buffers* bufs,
   if (cudaGetDevice(&device) != cudaSuccess) return KIVI_ERR_CUDA;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
     return KIVI_ERR_CUDA;
-  if (cudaMemset(bufs->workspace, 0, kivi::kWsHeader) != cudaSuccess) return KIVI_ERR_CUDA;
+  // status word and tickets start at zero (the decode kernel leaves the tickets at zero)
+  const size_t clear = kivi::kWsHeader +
+                       kivi::ws_tickets_bytes((long)cfg->batch * cfg->num_kv_heads);
+  if (cudaMemset(bufs->workspace, 0, clear) != cudaSuccess) return KIVI_ERR_CUDA;
   kivi_cache* h = new (std::nothrow) kivi_cache();
   if (!h) return KIVI_ERR_INVALID_ARG;
   h->cfg = *cfg;
@@ -129,7 +148,6 @@ kivi_status kivi_cache_create(const kivi_config* cfg, const kivi_buffers* bufs,
   h->S.assign(cfg->num_layers, 0);
   h->ngcap = kivi::num_groups(cfg->max_tokens);
   h->rec_bytes = record_bytes(cfg);
-  h->max_splits = kivi::max_splits(cfg->batch, cfg->num_kv_heads);
   h->num_sms = sms;
   h->device = device;
   *out = h;
@@ -222,19 +240,15 @@ kivi_status kivi_decode_attention(const kivi_cache* cache, int32_t layer, const 
   a.ring_v = layer_ring(cache, cache->bufs.resid_v, layer);
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.out = out;
-  uint8_t* ws = static_cast<uint8_t*>(cache->bufs.workspace);
-  const size_t parts = (size_t)cache->cfg.batch * cache->cfg.num_q_heads * cache->max_splits;
-  a.status = reinterpret_cast<uint32_t*>(ws);
-  a.ws_ml = reinterpret_cast<float*>(ws + kivi::kWsHeader);
-  a.ws_acc = a.ws_ml + 2 * parts;
+  bind_workspace(a, &cache->cfg, cache->bufs.workspace, cache->bufs.sizes.workspace_bytes);
   a.B = cache->cfg.batch;
   a.Hkv = cache->cfg.num_kv_heads;
   a.Hq = cache->cfg.num_q_heads;
   a.S = cache->S[layer];
   a.ngcap = cache->ngcap;
   a.sm_scale = sm_scale;
-  a.max_splits = cache->max_splits;
   a.num_sms = cache->num_sms;
+  a.device = cache->device;
   return from_cuda(kivi::launch_decode(cache->cfg.head_dim, cache->cfg.bits, a,
                                        static_cast<cudaStream_t>(stream)));
 }
@@ -247,7 +261,11 @@ kivi_status kivi_check_device_status(kivi_cache* cache, void* stream, uint32_t* 
   if (cudaMemcpy(&code, cache->bufs.workspace, sizeof code, cudaMemcpyDeviceToHost) !=
       cudaSuccess)
     return KIVI_ERR_CUDA;
-  if (code != 0 && cudaMemset(cache->bufs.workspace, 0, sizeof code) != cudaSuccess)
+  // after a failure the tickets may be left counting: clear them with the word
+  const size_t clear =
+      kivi::kWsHeader +
+      kivi::ws_tickets_bytes((long)cache->cfg.batch * cache->cfg.num_kv_heads);
+  if (code != 0 && cudaMemset(cache->bufs.workspace, 0, clear) != cudaSuccess)
     return KIVI_ERR_CUDA;
   if (code_out) *code_out = code;
   return code ? KIVI_ERR_DEVICE : KIVI_OK;
@@ -300,18 +318,20 @@ static __device__ __align__(256) unsigned char g_kivi_static_scratch[KIVI_STATIC
 
 namespace {
 
-constexpr int kMaxDevices = 64;
+using kivi::kMaxDevices;
 
 struct StaticScratchSlot {
   void* ptr = nullptr;  // device address of g_kivi_static_scratch on this device
   int num_sms = 0;
+  int device = 0;
 };
 
 std::mutex g_static_mu;
 StaticScratchSlot g_static_slots[kMaxDevices];
 
 // Once per device, with that device current: look up the array's address and
-// clear its header on `stream` (the status word must start at zero).
+// clear the whole array on `stream` (the status word and the tickets of any
+// shape must start at zero; the decode kernel leaves the tickets at zero).
 kivi_status static_scratch_slot(cudaStream_t stream, StaticScratchSlot* out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KIVI_ERR_CUDA;
@@ -324,9 +344,11 @@ kivi_status static_scratch_slot(cudaStream_t stream, StaticScratchSlot* out) {
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return KIVI_ERR_CUDA;
-    if (cudaMemsetAsync(p, 0, kivi::kWsHeader, stream) != cudaSuccess) return KIVI_ERR_CUDA;
+    if (cudaMemsetAsync(p, 0, KIVI_STATIC_SCRATCH_BYTES, stream) != cudaSuccess)
+      return KIVI_ERR_CUDA;
     slot.ptr = p;
     slot.num_sms = sms;
+    slot.device = dev;
   }
   *out = slot;
   return KIVI_OK;
@@ -350,20 +372,23 @@ extern "C" kivi_status kivi_decode_attention_static_scratch(
   if (S < 0) return KIVI_ERR_INVALID_ARG;
   if (S == 0) return KIVI_ERR_STATE;
   if (S > cfg->max_tokens) return KIVI_ERR_CAPACITY;
-  const size_t rows = (size_t)cfg->batch * cfg->num_q_heads;
-  const size_t per_split = rows * (2 + (size_t)cfg->head_dim) * sizeof(float);
-  // at least one split over the quantized groups plus the residual chunks
-  if (kivi::kWsHeader + kivi::kMinSplits * per_split > KIVI_STATIC_SCRATCH_BYTES)
-    return KIVI_ERR_SCRATCH_LIMIT;
-  const int fit = (int)((KIVI_STATIC_SCRATCH_BYTES - kivi::kWsHeader) / per_split);
-  const int max_splits = std::min(kivi::max_splits(cfg->batch, cfg->num_kv_heads), fit);
+  const long pairs = (long)cfg->batch * cfg->num_kv_heads;
+  const int hpk = cfg->num_q_heads / cfg->num_kv_heads;
+
+  // the fixed part (status word, tickets) must fit before any device work
+  const long fixed = kivi::kWsHeader + kivi::ws_tickets_bytes(pairs);
+  if (fixed + partial_bytes(cfg) > (long)KIVI_STATIC_SCRATCH_BYTES) return KIVI_ERR_SCRATCH_LIMIT;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   StaticScratchSlot slot;
   st = static_scratch_slot(s, &slot);
   if (st != KIVI_OK) return st;
+  const int grid = kivi::decode_grid_ctas(cfg->head_dim, cfg->bits, hpk, pairs, S, slot.num_sms);
+  if (grid < 1) return KIVI_ERR_UNSUPPORTED;
+  if (fixed + grid * partial_bytes(cfg) > (long)KIVI_STATIC_SCRATCH_BYTES)
+    return KIVI_ERR_SCRATCH_LIMIT;
 
-  const size_t seqs = (size_t)cfg->batch * cfg->num_kv_heads;
+  const size_t seqs = (size_t)pairs;
   const long rb = record_bytes(cfg);
   kivi::DecodeArgs a;
   a.records = static_cast<const uint8_t*>(records) + (size_t)layer * seqs * ngcap * rb;
@@ -373,17 +398,30 @@ extern "C" kivi_status kivi_decode_attention_static_scratch(
              (size_t)layer * seqs * kRingSlots * cfg->head_dim;
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.out = out;
-  uint8_t* ws = static_cast<uint8_t*>(slot.ptr);
-  a.status = reinterpret_cast<uint32_t*>(ws);
-  a.ws_ml = reinterpret_cast<float*>(ws + kivi::kWsHeader);
-  a.ws_acc = a.ws_ml + 2 * rows * max_splits;
+  bind_workspace(a, cfg, slot.ptr, KIVI_STATIC_SCRATCH_BYTES);
   a.B = cfg->batch;
   a.Hkv = cfg->num_kv_heads;
   a.Hq = cfg->num_q_heads;
   a.S = S;
   a.ngcap = ngcap;
   a.sm_scale = sm_scale;
-  a.max_splits = max_splits;
   a.num_sms = slot.num_sms;
+  a.device = slot.device;
   return from_cuda(kivi::launch_decode(cfg->head_dim, cfg->bits, a, s));
+}
+
+extern "C" kivi_status kivi_static_scratch_status(void* stream, uint32_t* code_out) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  StaticScratchSlot slot;
+  kivi_status st = static_scratch_slot(s, &slot);
+  if (st != KIVI_OK) return st;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return KIVI_ERR_CUDA;
+  uint32_t code = 0;
+  if (cudaMemcpy(&code, slot.ptr, sizeof code, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return KIVI_ERR_CUDA;
+  // after a failure the tickets may be left counting: clear the whole array
+  if (code != 0 && cudaMemset(slot.ptr, 0, KIVI_STATIC_SCRATCH_BYTES) != cudaSuccess)
+    return KIVI_ERR_CUDA;
+  if (code_out) *code_out = code;
+  return code ? KIVI_ERR_DEVICE : KIVI_OK;
 }

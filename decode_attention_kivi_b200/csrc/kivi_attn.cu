@@ -2,35 +2,51 @@
 //
 // For query head h of sequence b (kv head h / (Hq/Hkv)), over all S cached tokens:
 //   s_t = sm_scale * <q, k_t>,  out = sum_t softmax(s)_t v_t,
-// where k_t, v_t are the dequantized codes (scale_h * code + min_h) for the
+// where k_t, v_t are the dequantized codes (scale_h * code + min_h) of the
 // NG(S)*32 grouped tokens and the bf16 residual ring for the rest (record
 // "kv-efficiency/kivi-2bit-llama3-8b-gqa-8k", "KV bytes basis": the most recent
 // R tokens stay full precision).  Grouped history and residual share one
 // online softmax.
 //
-// Group CTAs (split < splits_g of each sequence and kv head; one wave of 4 CTAs
-// per SM): each warp streams whole 32-token group
-// records (one contiguous block each) into its own shared-memory ring with
-// cp.async.bulk on mbarriers, and does both contractions on the tensor cores
-// (mma.sync m16n8k16, fp16 operands, fp32 accumulation):
+// Work: one persistent CTA per SM.  The work of a (sequence, kv head) pair is a
+// list of items: pairs of group records (64 tokens), a last single record, and
+// residual items of 8 ring tokens.  The items of all pairs, in order, are split
+// into one contiguous range per CTA, balanced by their bytes; inside a CTA the
+// warps claim items from a shared counter, so warps that run ahead take more.
+// Each warp streams its items into its own two-item shared-memory ring with
+// cp.async.bulk on mbarriers and keeps one online-softmax state per pair; when
+// it moves to another pair it merges that state into the CTA's slot for the
+// pair.  At the end each CTA writes the output of the pairs it holds whole; for
+// a pair shared with other CTAs it writes a partial, and the last CTA to
+// arrive (a ticket per pair) merges the partials into the output.
+//
+// Group records, on the tensor cores (mma.sync m16n8k16, fp16 operands, fp32
+// accumulation):
 //   scores  C[token][head] = sum_d code[token][d] * (q''[head][d] * kscale[d])
 //                          + sum_d kmin[d] * q''[head][d]
-//           with q'' * kscale carried as an fp16 pair hi + lo (two MMAs sharing
-//           the code operand) so the scores keep about 22 significant bits
+//           with q'' * kscale carried as an fp16 pair hi + lo (the two halves of
+//           the exact product of two fp16 numbers) in adjacent columns;
 //   P.V     C[chan][head] += sum_t code[t][chan] * (p[head][t] * vscale[t][j])
 //                          + sum_t vmin[t][j] * p[head][t]
-// The codes become exact fp16 small integers with one three-input logic op and
-// one add per pair (the packing puts adjacent codes in the two halves of a word); the
-// scale and the min fold into the other operand, so nothing is dequantized
-// element by element.  The min terms are MMAs whose A rows all repeat the min
-// vector.  q'' = q * 2^-e_h (exact) keeps |q''| < 1 so q'' * kscale stays in
-// fp16 range; scores are rescaled by 2^e_h * sm_scale * log2(e) in fp32.
+//           with p * vscale carried as hi + lo as well: p is split into fp16
+//           hi + lo, and for up to four heads per kv head the lo parts use the
+//           four columns the heads leave free.
+// The codes turn into exact fp16 operands with the sm_100a conversions of
+// packed small floats: one mask spreads eight 2-bit codes into nibbles, and one
+// conversion turns a byte of two nibbles into two fp16 values c/2 (4-bit codes:
+// a byte holds one code, the value is c/8).  The scale and the min fold into
+// the other operand, so nothing is dequantized element by element; the
+// constant factor 1/2 (1/8) is undone in fp32.  q'' = q * 2^-e_h (exact) keeps
+// |q''| < 1 so q'' * kscale stays in fp16 range; scores are rescaled by
+// 2^e_h * sm_scale * log2(e) in fp32.
 //
-// Residual-chunk CTAs (after the group CTAs in the grid; they fill the SMs the
-// group CTAs leave free): 32 bf16 ring tokens each, on CUDA cores.
-// Every CTA writes one (m, l, acc) partial per query head; combine_kernel
-// merges the partials.  Every wait on an mbarrier is bounded; a wait that runs
-// out sets the device status word and the CTA stops issuing work.
+// Residual items: 8 bf16 ring tokens on the tensor cores in bf16 (exact
+// products): scores with q itself, P.V with p as a bf16 hi + lo pair in the two
+// halves of the k dimension.
+//
+// Every wait is bounded: a wait on an mbarrier or a lock that runs out sets the
+// device status word and the warp stops issuing work; the CTA still finishes
+// its bookkeeping so that no other CTA waits on it.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -41,17 +57,16 @@
 namespace kivi {
 namespace {
 
-constexpr int kWarps = 4;
-constexpr int kThreads = kWarps * 32;
-constexpr int kStages = 4;
-// Row stride (fp16 entries) of a warp's p tile [8 heads][64 tokens]: 64 plus 8 of
-// padding, so that the eight rows a P.V operand load touches fall in distinct
-// banks (a 64-entry row is 128 bytes: every row would start in bank 0).
-constexpr int kPRow = 2 * 32 + 8;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr long long kWaitBudgetCycles = 4000000000LL;  // about 2 s at 1.9 GHz
+constexpr int kLockSpinLimit = 1 << 24;
 constexpr uint32_t kStatusWaitTimeout = 1u;
-constexpr int kMaxResidualChunks = (kRingSlots + kGroup - 1) / kGroup;  // residual < R + G tokens
+constexpr uint32_t kStatusLockTimeout = 2u;
+constexpr uint32_t kStatusBadSplit = 4u;
+constexpr int kResTok = 8;             // residual tokens per item
+constexpr int kPRow = 2 * 32 + 8;      // p tile row (fp16 entries): 64 tokens + 8 padding
+constexpr int kGridBase = 256;         // CTAs at most, before the pair-slot bound
+constexpr int kSmemBudget = 227 * 1024;
 
 // ---------------------------------------------------------------------------
 // PTX wrappers
@@ -117,11 +132,30 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
 
 __device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                         uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
       "{%8,%9}, {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
 }
 
 __device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
@@ -136,75 +170,22 @@ __device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
   return d;
 }
 
+// (a & b) | c and (a & b) ^ c as one three-input logic op each.
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ uint32_t and_xor(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   const __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&h);
 }
-
-// ---------------------------------------------------------------------------
-// Codes -> exact fp16 pairs
-// ---------------------------------------------------------------------------
-
-// The two codes at bit offset P of each 16-bit half of w, as fp16x2 (c_lo, c_hi).
-// OR-ing the masked bits under the fp16 exponent of 2^(10-P) puts the code bits
-// at weight 1: the half is 2^(10-P) + c exactly (P + BITS <= 10), and one add
-// of -2^(10-P) leaves c.  The magic constants live in registers (CodeConsts).
-template <int BITS>
-struct CodeConsts {
-  static constexpr int kNumP = BITS == 2 ? 5 : 2;  // offsets P = 0, b, 2b, ... below 10
-  uint32_t magic[kNumP];                           // fp16x2 2^(10-P)
-  uint32_t neg[kNumP];                             // fp16x2 -2^(10-P)
-  __device__ __forceinline__ void init() {
-#pragma unroll
-    for (int i = 0; i < kNumP; ++i) {
-      const uint32_t e = (uint32_t)(25 - i * BITS) << 10;
-      magic[i] = e | (e << 16);
-      neg[i] = magic[i] | 0x80008000u;
-      // opaque to the compiler: keep the constants in registers instead of
-      // rematerializing them at every use
-      asm volatile("" : "+r"(magic[i]), "+r"(neg[i]));
-    }
-  }
-};
-
-__device__ __forceinline__ uint32_t hadd2(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-
-// (w & mask) | magic as one three-input logic op (LUT 0xEA = (a & b) | c); the
-// two-operator C form costs two instructions.
-template <uint32_t MASK>
-__device__ __forceinline__ uint32_t and_or(uint32_t w, uint32_t magic) {
-  uint32_t d;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(w), "n"(MASK), "r"(magic));
-  return d;
-}
-
-template <int BITS, int P>
-__device__ __forceinline__ uint32_t code_pair(uint32_t w, const CodeConsts<BITS>& k) {
-  static_assert(P + BITS <= 10 && P % BITS == 0, "code bits must lie inside the fp16 mantissa");
-  constexpr uint32_t m = ((1u << BITS) - 1u) << P;
-  return hadd2(and_or<m | (m << 16)>(w, k.magic[P / BITS]), k.neg[P / BITS]);
-}
-
-// Pair K (codes 2K and 2K+1) of a word; pairs past the fp16 mantissa come from
-// the word shifted right by kHiShift.
-template <int BITS>
-struct CodeWord {
-  static constexpr int kHiShift = BITS == 2 ? 10 : 8;
-  template <int K>
-  static __device__ __forceinline__ uint32_t pair(uint32_t w, uint32_t w_hi,
-                                                  const CodeConsts<BITS>& k) {
-    constexpr int off = K * BITS;
-    if constexpr (off + BITS <= 10) {
-      return code_pair<BITS, off>(w, k);
-    } else {
-      return code_pair<BITS, off - kHiShift>(w_hi, k);
-    }
-  }
-};
 
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
@@ -213,693 +194,1023 @@ __device__ __forceinline__ float fast_exp2(float x) {
 }
 
 // ---------------------------------------------------------------------------
-// Shared memory plan (dynamic)
+// Codes -> exact fp16 operands
 // ---------------------------------------------------------------------------
 
+// Byte K of x holds two e2m1 values (2-bit codes in the low bits of its
+// nibbles): fp16x2 (low nibble / 2, high nibble / 2).
+template <int K>
+__device__ __forceinline__ uint32_t e2m1_byte(uint32_t x) {
+  uint32_t d;
+  if constexpr (K == 0)
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t}" : "=r"(d) : "r"(x));
+  else if constexpr (K == 1)
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b1;\n\t}" : "=r"(d) : "r"(x));
+  else if constexpr (K == 2)
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b2;\n\t}" : "=r"(d) : "r"(x));
+  else
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b3;\n\t}" : "=r"(d) : "r"(x));
+  return d;
+}
+
+// Half-word K of x holds two e2m3 values (4-bit codes in the low nibbles of its
+// bytes): fp16x2 (low byte / 8, high byte / 8).
+template <int K>
+__device__ __forceinline__ uint32_t e2m3_half(uint32_t x) {
+  uint32_t d;
+  if constexpr (K == 0)
+    asm("{\n\t.reg .b16 h0, h1;\n\tmov.b32 {h0, h1}, %1;\n\t"
+        "cvt.rn.f16x2.e2m3x2 %0, h0;\n\t}" : "=r"(d) : "r"(x));
+  else
+    asm("{\n\t.reg .b16 h0, h1;\n\tmov.b32 {h0, h1}, %1;\n\t"
+        "cvt.rn.f16x2.e2m3x2 %0, h1;\n\t}" : "=r"(d) : "r"(x));
+  return d;
+}
+
+// A operands of k-step SL of a K-code word pair (rows g and g + 8): a0..a3,
+// from the words already masked into nibbles (2 bits: m0 = w & 0x33333333 and
+// m2 = (w >> 2) & 0x33333333; 4 bits: m0 = w & 0x0F0F0F0F, m2 = (w >> 4) & ...).
+template <int BITS, int SL>
+__device__ __forceinline__ void key_operands(uint32_t m0, uint32_t m2, uint32_t n0, uint32_t n2,
+                                             uint32_t (&a)[4]) {
+  if constexpr (BITS == 2) {
+    // byte SL: codes j = 0 (bits 0-1), 1 (4-5) -> a0; j = 2 (2-3), 3 (6-7) -> a2
+    a[0] = e2m1_byte<SL>(m0);
+    a[2] = e2m1_byte<SL>(m2);
+    a[1] = e2m1_byte<SL>(n0);
+    a[3] = e2m1_byte<SL>(n2);
+  } else {
+    // nibble SL of every byte j: half-word 0 -> (j0, j1) = a0, half-word 1 -> a2
+    const uint32_t x = SL == 0 ? m0 : m2, y = SL == 0 ? n0 : n2;
+    a[0] = e2m3_half<0>(x);
+    a[2] = e2m3_half<1>(x);
+    a[1] = e2m3_half<0>(y);
+    a[3] = e2m3_half<1>(y);
+  }
+}
+
+template <int BITS>
+__device__ __forceinline__ void key_masks(uint32_t w, uint32_t& m0, uint32_t& m2) {
+  if constexpr (BITS == 2) {
+    m0 = w & 0x33333333u;
+    m2 = (w >> 2) & 0x33333333u;
+  } else {
+    m0 = w & 0x0F0F0F0Fu;
+    m2 = (w >> 4) & 0x0F0F0F0Fu;
+  }
+}
+
+// A operands (a0..a3) of k-step kk of V-code m-tile: 2 bits from lane word x
+// (both k-steps), 4 bits from the k-step's own word.
+template <int BITS>
+__device__ __forceinline__ void value_operands(uint32_t x, int kk, uint32_t (&a)[4]) {
+  if constexpr (BITS == 2) {
+    const uint32_t y = (x >> (2 * kk)) & 0x33333333u;  // byte r + 2 hf
+    a[0] = e2m1_byte<0>(y);
+    a[1] = e2m1_byte<1>(y);
+    a[2] = e2m1_byte<2>(y);
+    a[3] = e2m1_byte<3>(y);
+  } else {
+    const uint32_t lo = x & 0x0F0F0F0Fu, hi = (x >> 4) & 0x0F0F0F0Fu;  // r = 0, 1
+    a[0] = e2m3_half<0>(lo);
+    a[2] = e2m3_half<1>(lo);
+    a[1] = e2m3_half<0>(hi);
+    a[3] = e2m3_half<1>(hi);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Configuration and shared-memory plan
+// ---------------------------------------------------------------------------
+
+__host__ __device__ constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
+__host__ __device__ constexpr int cmin_i(int a, int b) { return a < b ? a : b; }
+
 template <int D, int BITS, int HPK>
-struct Plan {
+struct Cfg {
   static constexpr RecordGeom geo{D, BITS};
-  static constexpr int kRec = (int)geo.bytes();             // bytes, multiple of 128
-  static constexpr int kStageBytes = kWarps * kStages * kRec;
-  static constexpr int kPBytes = kWarps * 8 * kPRow * 2;  // per warp p[8 heads][kPRow] fp16
-  static constexpr int kQBytes = HPK * D * 4;               // q (fp32) of this kv head
-  static constexpr int kMergeBytes = kWarps * HPK * D * 4;  // aliases the stages
-  static_assert(kMergeBytes <= kStageBytes, "merge area must fit in the stage area");
-  static constexpr int kResidPBytes = kWarps * HPK * kGroup * 4;  // residual p, aliases stages
-  static_assert(kResidPBytes <= kStageBytes, "residual scratch must fit in the stage area");
-  static constexpr int kOffP = kStageBytes;
-  static constexpr int kOffQ = kOffP + kPBytes;
-  static constexpr int kOffML = kOffQ + kQBytes;               // wm, wl [kWarps][8] each
-  static constexpr int kOffBar = kOffML + 2 * kWarps * 8 * 4;  // [kWarps][kStages] mbarriers
-  static constexpr int kBytes = kOffBar + kWarps * kStages * 8;
+  static constexpr int kRec = (int)geo.bytes();          // multiple of 128
+  static constexpr int kItemBytes = 2 * kRec;             // two records, or 8 K + 8 V rows
+  static constexpr int kResRow = 2 * D + 16;              // padded residual row (bank spread)
+  static_assert(kResTok * kResRow <= kRec, "residual rows must fit in one record's space");
+  static constexpr int kChunks = HPK > 4 ? 2 : 1;         // score column chunks of 4 heads
+  static constexpr bool kLoCols = HPK <= 4;               // P.V lo parts in the free columns
+  static constexpr int kCodeShift = BITS == 2 ? 1 : 3;    // operands are code / 2^shift
+  // p tile rows: heads' p_hi, then -p_lo (<= 4 heads) or p_lo (8 heads), then a zero row
+  static constexpr int kPRows = 2 * HPK + (kLoCols ? 1 : 0);
+  static constexpr int kZeroRow = 2 * HPK;
+  static constexpr int kWarpBytes = round_up(2 * kItemBytes + kPRows * kPRow * 2, 128);
+  static constexpr int kSlotBytes = round_up(96 + HPK * D * 4 + HPK * D * 2, 16);  // merge + q
+  static constexpr int kMinSlots = 4;
+  static constexpr int kFixed = 512;                      // mbarriers (16 B a warp), counter
+  static constexpr int kNW =
+      HPK > 4 ? 8 : cmin_i(16, (kSmemBudget - kFixed - kMinSlots * kSlotBytes) / kWarpBytes);
+  static constexpr int kThreads = kNW * 32;
+  static constexpr int kSlots =
+      cmin_i(64, (kSmemBudget - kFixed - kNW * kWarpBytes) / kSlotBytes);
+  static_assert(kNW >= 4 && kSlots >= kMinSlots, "shared-memory plan");
+  static_assert(16 * kNW + 8 <= kFixed, "mbarriers and the claim counter fit the fixed area");
+  static constexpr int kOffSlots = kNW * kWarpBytes;
+  static constexpr int kOffFixed = kOffSlots + kSlots * kSlotBytes;
+  static constexpr int kBytes = kOffFixed + kFixed;
+  // item costs for the split between CTAs: bytes read / 512 + 1
+  static constexpr int kCostG2 = 2 * kRec / 512 + 1;
+  static constexpr int kCostG1 = kRec / 512 + 1;
+  static constexpr int kCostR = kResTok * D * 4 / 512 + 1;
 };
+
+// One pair slot of a CTA: merged online-softmax state and the pair's q.
+template <int D, int HPK>
+struct PairSlot {
+  float m[8];
+  float l[8];
+  int lock;
+  int pad[7];
+  float acc[HPK][D];
+  __nv_bfloat16 q[HPK][D];
+};
+
+// ---------------------------------------------------------------------------
+// The split of the items between CTAs
+// ---------------------------------------------------------------------------
+
+// Items of one pair: n2 record pairs, n1 (0 or 1) single record, nr residual
+// items; costs c2, c1, cr.  The CTA ranges cut the concatenated cost axis of
+// all pairs into n equal parts: CTA c owns [lo(c), lo(c+1)) with
+// lo(c) = c*q + min(c, rem), and the items whose cost interval starts there.
+struct Split {
+  int pairs, ipp, n2, n1, nr, NG;
+  int c2, c1, cr, pc;  // item costs, cost per pair
+  int n, q, rem;       // CTAs and the division of pairs*pc among them
+};
+
+__host__ __device__ inline int cost_lo(const Split& s, int c) {
+  return c * s.q + (c < s.rem ? c : s.rem);
+}
+
+__host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// First item whose cost interval starts at or after cost x (global item index).
+__host__ __device__ inline int first_item_at(const Split& s, int x) {
+  const int p = x / s.pc, w = x % s.pc;
+  int k;
+  if (w <= s.n2 * s.c2) {
+    k = ceil_div(w, s.c2);
+  } else if (w <= s.n2 * s.c2 + s.n1 * s.c1) {
+    k = s.n2 + ceil_div(w - s.n2 * s.c2, s.c1);
+  } else {
+    k = s.n2 + s.n1 + ceil_div(w - s.n2 * s.c2 - s.n1 * s.c1, s.cr);
+  }
+  return p * s.ipp + k;  // k == ipp is item 0 of pair p + 1
+}
+
+__host__ __device__ inline int cta_first_item(const Split& s, int c) {
+  return first_item_at(s, cost_lo(s, c));
+}
+
+// The CTA that owns global item `it`.
+__host__ __device__ inline int cta_of_item(const Split& s, int it) {
+  const int p = it / s.ipp, k = it % s.ipp;
+  int cs = p * s.pc;
+  if (k <= s.n2) cs += k * s.c2;
+  else if (k <= s.n2 + s.n1) cs += s.n2 * s.c2 + (k - s.n2) * s.c1;
+  else cs += s.n2 * s.c2 + s.n1 * s.c1 + (k - s.n2 - s.n1) * s.cr;
+  const int big = s.rem * (s.q + 1);
+  return cs < big ? cs / (s.q + 1) : s.rem + (cs - big) / s.q;
+}
 
 // ---------------------------------------------------------------------------
 // The decode kernel
 // ---------------------------------------------------------------------------
 
 template <int D, int BITS, int HPK>
-__global__ void __launch_bounds__(kThreads, HPK <= 4 ? 4 : 2)
-decode_kernel(DecodeArgs args, int splits_g, int n_res, int groups_per_cta, float qscale) {
-  // Linear grid: B*Hkv*splits_g group CTAs (split fastest), then B*Hkv*n_res
-  // residual-chunk CTAs, which take the slots the group CTAs leave free.
-  using P = Plan<D, BITS, HPK>;
-  using CW = CodeWord<BITS>;
-  constexpr RecordGeom geo = P::geo;
-  constexpr int kKSteps = D / 16;            // score k-steps (16 channels each)
-  constexpr int kMTiles = D / 16;            // P.V m-tiles (16 channels each)
-  constexpr int kBlocks = D / 32;            // value channel blocks j
-  constexpr int kThrWords = D * BITS / 128;  // K-code words one thread reads per token row
-  constexpr int kChunks = HPK > 4 ? 2 : 1;   // score column chunks of 4 heads x {hi, lo}
-  constexpr int kVWords = kMTiles * BITS / 2;  // V-code words one thread reads per group
+struct Warp;  // per-warp state and item processing (below)
 
-  extern __shared__ __align__(128) unsigned char smem[];
-  float* q_s = reinterpret_cast<float*>(smem + P::kOffQ);
-  float* wm = reinterpret_cast<float*>(smem + P::kOffML);
-  float* wl = wm + kWarps * 8;
+template <int D, int BITS, int HPK>
+struct Warp {
+  using C = Cfg<D, BITS, HPK>;
+  static constexpr RecordGeom geo = C::geo;
+  static constexpr int kChunks = C::kChunks;
+  static constexpr int kKSteps = D / 16;             // score k-steps (16 channels each)
+  static constexpr int kMTiles = D / 16;             // P.V m-tiles (16 channels each)
+  static constexpr int kBlocks = D / 32;             // value channel blocks j
+  static constexpr int kLaneWordsK = D * BITS / 128;  // K-code words of one quad lane per row
+  static constexpr int kStepsPerWord = 8 / BITS;
+  static constexpr int kVWords = kMTiles * BITS / 2;  // V-code words of one lane per record
 
-  const int n_group_ctas = splits_g * args.Hkv * args.B;
-  int split, kvh, b;
-  if ((int)blockIdx.x < n_group_ctas) {
-    split = blockIdx.x % splits_g;
-    kvh = (blockIdx.x / splits_g) % args.Hkv;
-    b = blockIdx.x / (splits_g * args.Hkv);
-  } else {
-    const int r = blockIdx.x - n_group_ctas;
-    split = splits_g + r % n_res;
-    kvh = (r / n_res) % args.Hkv;
-    b = r / (n_res * args.Hkv);
-  }
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int Hq = args.Hq, S = args.S;
-  const long seq = (long)b * args.Hkv + kvh;
-  const int NG = num_groups(S);
+  const DecodeArgs& a;
+  const int lane, g, tig;
+  // online softmax state of the current pair: heads 4c + tig
+  float m_run[kChunks], l_run[kChunks];
+  float acc[kMTiles][4];  // (channel 16mt + g (+8), column 2tig + e)
+  float vmacc[4];         // value-min term: (row g -> block g % kBlocks, column 2tig + e)
+  // score B operands of the current pair: q'' split so that one fma gives hi or lo
+  uint32_t qa[kChunks][kKSteps][2], qb[kChunks][kKSteps][2];
+  float ch[kChunks];      // log2 score scale of head 4c + tig
+  float qscale;           // sm_scale * log2(e)
+  const __nv_bfloat16* q_pair;  // the pair's q (HPK x D) in shared memory
+  unsigned char* p_tile;  // this warp's p tile
+  int rowA, rowX, rowR;   // p tile rows this lane reads (byte offsets)
+  uint32_t maskY, signY, maskHi;
 
-  const bool group_cta = split < splits_g;
-  const int g = lane >> 2, tig = lane & 3;
-  float* merge_acc = reinterpret_cast<float*>(smem);  // [kWarps][HPK][D], used after the loop
-  // Group-CTA geometry: this warp's groups are first + warp, first + warp + kWarps, ...
-  unsigned char* stage0 = smem + warp * kStages * P::kRec;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P::kOffBar) + warp * kStages;
-  __half* p_s = reinterpret_cast<__half*>(smem + P::kOffP) + warp * 8 * kPRow;
-  const int first = split * groups_per_cta;
-  const int last = min(NG, first + groups_per_cta);
-  const int n_mine =
-      group_cta && first + warp < last ? (last - first - warp + kWarps - 1) / kWarps : 0;
-  const uint8_t* seq_rec = args.records + seq * args.ngcap * (long)P::kRec;
-  if (group_cta) {
-    for (int i = lane; i < 8 * kPRow / 2; i += 32)
-      reinterpret_cast<uint32_t*>(p_s)[i] = 0u;  // heads without a query stay finite
-    if (lane == 0) {
-      for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
-      fence_mbar_init();
-    }
-  }
+  __device__ Warp(const DecodeArgs& args, int lane_, float qs)
+      : a(args), lane(lane_), g(lane_ >> 2), tig(lane_ & 3), qscale(qs) {}
 
-  wait_for_predecessor();  // q, the records and the rings may come from the previous kernel
-  // q of this kv head's query heads (16-byte pieces): the loads go out before
-  // the record stream so that they do not queue behind it
-  constexpr int kQPieces = HPK * D / 8;
-  static_assert(kQPieces <= kThreads, "one 16-byte piece of q per thread");
-  uint4 qv = make_uint4(0u, 0u, 0u, 0u);
-  if (threadIdx.x < kQPieces)  // the heads of kv head kvh are contiguous
-    qv = reinterpret_cast<const uint4*>(args.q + ((long)b * Hq + kvh * HPK) * D)[threadIdx.x];
-  if (group_cta && lane == 0) {
-    for (int i = 0; i < kStages && i < n_mine; ++i) {
-      mbar_expect_tx(&bars[i], P::kRec);
-      bulk_load(stage0 + i * P::kRec, seq_rec + (long)(first + warp + i * kWarps) * P::kRec,
-                P::kRec, &bars[i]);
-    }
-  }
-  if (threadIdx.x < kQPieces) {  // q as fp32 in smem
-    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&qv);
-    float4* dst = reinterpret_cast<float4*>(q_s + threadIdx.x * 8);
-    const float2 f0 = __bfloat1622float2(h2[0]), f1 = __bfloat1622float2(h2[1]);
-    const float2 f2 = __bfloat1622float2(h2[2]), f3 = __bfloat1622float2(h2[3]);
-    dst[0] = make_float4(f0.x, f0.y, f1.x, f1.y);
-    dst[1] = make_float4(f2.x, f2.y, f3.x, f3.y);
-  }
-  __syncthreads();
-
-  if (group_cta) {
-    // ===================== group CTA: tensor-core path =====================
-    CodeConsts<BITS> kc;
-    kc.init();
-
-    // Score B operand: column n = g is head 4c + g/2 of chunk c, hi part for even
-    // g and lo part for odd g.  qq = q''[head][channels c0..c0+3] per k-step,
-    // c0 = tig*D/4 + 4s.  negm = -1 (odd g) or 0 (even g) in fp16x2.
-    // Per-head exponent e_h with max |q_h| 2^-e_h in [0.5, 1), computed by every
-    // warp: lanes [h L, (h+1) L) take head h (L = 32 / HPK lanes, D / L values each).
-    int ex[HPK];
-    {
-      constexpr int kLanesPerHead = 32 / HPK;
-      constexpr int kPerLane = D / kLanesPerHead;
-      const float* qh = q_s + (lane / kLanesPerHead) * D + (lane % kLanesPerHead) * kPerLane;
-      float mx = 0.f;
-#pragma unroll
-      for (int i = 0; i < kPerLane; ++i) mx = fmaxf(mx, fabsf(qh[i]));
-#pragma unroll
-      for (int o = 1; o < kLanesPerHead; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      int e = 0;
-      if (mx > 0.f) frexpf(mx, &e);
-#pragma unroll
-      for (int hh = 0; hh < HPK; ++hh) ex[hh] = __shfl_sync(0xffffffffu, e, hh * kLanesPerHead);
-    }
-    uint32_t qq[kChunks][kKSteps][2];
-    const uint32_t negm = (g & 1) ? 0xBC00BC00u : 0u;
-    float ch[kChunks];  // log2 score scale of head 4c + tig
-#pragma unroll
-    for (int c = 0; c < kChunks; ++c) {
-      const int hs = 4 * c + g / 2;
-      int es = 0, et = 0;
-#pragma unroll
-      for (int hh = 0; hh < HPK; ++hh) {
-        es = hh == hs ? ex[hh] : es;
-        et = hh == 4 * c + tig ? ex[hh] : et;
-      }
-#pragma unroll
-      for (int s = 0; s < kKSteps; ++s) {
-        const int c0 = tig * (D / 4) + 4 * s;
-        if (hs < HPK) {
-          const float sc = ldexpf(1.f, -es);
-          const float* qr = q_s + hs * D + c0;
-          qq[c][s][0] = pack_half2(qr[0] * sc, qr[1] * sc);
-          qq[c][s][1] = pack_half2(qr[2] * sc, qr[3] * sc);
-        } else {
-          qq[c][s][0] = qq[c][s][1] = 0u;
-        }
-      }
-      const int hh = 4 * c + tig;
-      ch[c] = hh < HPK ? ldexpf(qscale, et) : 1.f;  // > 0 keeps -inf scores at p = 0
-    }
-
-    float acc[kMTiles][4];
-    float vmacc[4] = {0.f, 0.f, 0.f, 0.f};  // sum_t vmin[t][j] p[h][t], row g -> block g % kBlocks
-#pragma unroll
-    for (int mt = 0; mt < kMTiles; ++mt)
-#pragma unroll
-      for (int r = 0; r < 4; ++r) acc[mt][r] = 0.f;
-    float m_run[kChunks], l_run[kChunks];
+  __device__ __forceinline__ void reset() {
 #pragma unroll
     for (int c = 0; c < kChunks; ++c) {
       m_run[c] = -INFINITY;
       l_run[c] = 0.f;
     }
-
-    bool timed_out = false;
-    int i_stop = n_mine;
-    for (int i = 0; i < n_mine; i += 2) {
-      const bool has_b = i + 1 < n_mine;
-      bool arrived = mbar_wait_bounded(&bars[i % kStages], (uint32_t)(i / kStages) & 1u);
-      if (has_b)
-        arrived = arrived && mbar_wait_bounded(&bars[(i + 1) % kStages],
-                                               (uint32_t)((i + 1) / kStages) & 1u);
-      if (!__all_sync(0xffffffffu, arrived)) {  // warp-uniform decision
-        timed_out = true;
-        i_stop = i;
-        break;
-      }
-      const unsigned char* recs[2] = {stage0 + (i % kStages) * P::kRec,
-                                      stage0 + ((has_b ? i + 1 : i) % kStages) * P::kRec};
-
-      // ---- key-min term of both groups: rows g <- group A, rows g+8 <- group B ----
-      float cmin[kChunks][4];
 #pragma unroll
-      for (int c = 0; c < kChunks; ++c)
+    for (int mt = 0; mt < kMTiles; ++mt)
 #pragma unroll
-        for (int r = 0; r < 4; ++r) cmin[c][r] = 0.f;
-      {
-        const __half* kmA = reinterpret_cast<const __half*>(recs[0] + geo.k_min_off());
-        const __half* kmB = reinterpret_cast<const __half*>(recs[1] + geo.k_min_off());
+      for (int r = 0; r < 4; ++r) acc[mt][r] = 0.f;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) vmacc[r] = 0.f;
+  }
+
+  // The pair's q (bf16 in shared memory): the score B operands and scales.
+  __device__ __forceinline__ void load_pair(const __nv_bfloat16* qs) {
+    q_pair = qs;
+    // per-head exponent e_h with max |q_h| 2^-e_h in [0.5, 1): lanes of head hs
+    // (g = 2hs', 2hs'+1 in chunk c) each scan the head's D/4 channels of quad lane tig
+    int e_h[kChunks];
+#pragma unroll
+    for (int c = 0; c < kChunks; ++c) {
+      const int hs = 4 * c + g / 2;
+      float mx = 0.f;
+      if (hs < HPK) {
 #pragma unroll
         for (int s = 0; s < kKSteps; ++s) {
-          const int c0 = tig * (D / 4) + 4 * s;
-          const uint2 a = *reinterpret_cast<const uint2*>(kmA + c0);
-          const uint2 bb = *reinterpret_cast<const uint2*>(kmB + c0);
-#pragma unroll
-          for (int c = 0; c < kChunks; ++c) mma_f16(cmin[c], a.x, bb.x, a.y, bb.y, qq[c][s][0], qq[c][s][1]);
+          const uint2 v = *reinterpret_cast<const uint2*>(qs + hs * D + 16 * s + 4 * tig);
+          const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.x));
+          const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.y));
+          mx = fmaxf(mx, fmaxf(fmaxf(fabsf(f0.x), fabsf(f0.y)), fmaxf(fabsf(f1.x), fabsf(f1.y))));
         }
       }
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      int e = 0;
+      if (mx > 0.f) frexpf(mx, &e);
+      e_h[c] = e;
+      const float sc = ldexpf(1.f, -e);
+      const bool lo = (g & 1) != 0;
+#pragma unroll
+      for (int s = 0; s < kKSteps; ++s) {
+        uint32_t qq0 = 0u, qq1 = 0u;
+        if (hs < HPK) {
+          const uint2 v = *reinterpret_cast<const uint2*>(qs + hs * D + 16 * s + 4 * tig);
+          const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.x));
+          const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.y));
+          qq0 = pack_half2(f0.x * sc, f0.y * sc);
+          qq1 = pack_half2(f1.x * sc, f1.y * sc);
+        }
+        // hi column: qa = 0, qb = q''  -> fma(0, ks, RN(q'' ks)) = hi
+        // lo column: qa = q'', qb = -q'' -> fma(q'', ks, -RN(q'' ks)) = lo
+        qa[c][s][0] = lo ? qq0 : 0u;
+        qa[c][s][1] = lo ? qq1 : 0u;
+        qb[c][s][0] = lo ? (qq0 ^ 0x80008000u) : qq0;
+        qb[c][s][1] = lo ? (qq1 ^ 0x80008000u) : qq1;
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < kChunks; ++c) {
+      // exponent of head 4c + tig: held by the lanes with g = 2 tig
+      const int e = __shfl_sync(0xffffffffu, e_h[c], 8 * tig);
+      ch[c] = 4 * c + tig < HPK ? ldexpf(qscale, e + C::kCodeShift) : 1.f;
+    }
+  }
 
-      // ---- scores: sc[grp][c][mt][row half] ----
-      float sc[2][kChunks][2][2];
+  // Shares of alpha for the accumulator columns 2tig + e of this lane.
+  __device__ __forceinline__ void col_factors(const float (&f)[kChunks], float (&out)[2]) const {
 #pragma unroll
-      for (int grp = 0; grp < 2; ++grp) {
-        const unsigned char* rec = recs[grp];
-        const __half* kscale = reinterpret_cast<const __half*>(rec + geo.k_scale_off());
-        uint32_t bq[kChunks][kKSteps][2];
+    for (int e = 0; e < 2; ++e) {
+      const int col = 2 * tig + e;
+      const int h = C::kLoCols ? (col & 3) : col;
+      const int src = (lane & ~3) | (h & 3);
+      float v = __shfl_sync(0xffffffffu, f[0], src);
+      if constexpr (kChunks == 2) {
+        const float v1 = __shfl_sync(0xffffffffu, f[kChunks - 1], src);
+        v = h >= 4 ? v1 : v;
+      }
+      out[e] = v;
+    }
+  }
+
+  __device__ __forceinline__ void rescale(const float (&alpha)[kChunks]) {
+    bool same = true;
 #pragma unroll
-        for (int s = 0; s < kKSteps; ++s) {
-          const int c0 = tig * (D / 4) + 4 * s;
-          const uint2 ks = *reinterpret_cast<const uint2*>(kscale + c0);
+    for (int c = 0; c < kChunks; ++c) same = same && alpha[c] == 1.f;
+    if (__all_sync(0xffffffffu, same)) return;
+    float al[2];
+    col_factors(alpha, al);
+#pragma unroll
+    for (int mt = 0; mt < kMTiles; ++mt) {
+      acc[mt][0] *= al[0];
+      acc[mt][1] *= al[1];
+      acc[mt][2] *= al[0];
+      acc[mt][3] *= al[1];
+    }
+    vmacc[0] *= al[0];
+    vmacc[1] *= al[1];
+    vmacc[2] *= al[0];
+    vmacc[3] *= al[1];
+  }
+
+  // Stores p (fp32, head 4c + tig, column col of the tile) as fp16 hi and
+  // (negated for <= 4 heads) lo.
+  __device__ __forceinline__ void store_p(int c, int col, float p) {
+    const int h = 4 * c + tig;
+    if (h >= HPK) return;
+    const __half hi = __float2half_rn(p);
+    const float r = C::kLoCols ? __half2float(hi) - p : p - __half2float(hi);
+    __half* t = reinterpret_cast<__half*>(p_tile) + col;
+    t[h * kPRow] = hi;
+    t[(HPK + h) * kPRow] = __float2half_rn(r);
+  }
+
+  __device__ __forceinline__ uint32_t lds32(const unsigned char* p) const {
+    return *reinterpret_cast<const uint32_t*>(p);
+  }
+
+  // MMAs of the k-steps SL.. of one K-code word pair into acc
+  template <int SL>
+  __device__ __forceinline__ void score_steps(uint32_t m0, uint32_t m2, uint32_t n0, uint32_t n2,
+                                              const uint32_t (&bq)[kChunks][kStepsPerWord][2],
+                                              float (&acc_)[kChunks][4]) {
+    if constexpr (SL < kStepsPerWord) {
+      uint32_t ka[4];
+      key_operands<BITS, SL>(m0, m2, n0, n2, ka);
+#pragma unroll
+      for (int c = 0; c < kChunks; ++c)
+        mma_f16(acc_[c], ka[0], ka[1], ka[2], ka[3], bq[c][SL][0], bq[c][SL][1]);
+      score_steps<SL + 1>(m0, m2, n0, n2, bq, acc_);
+    }
+  }
+
+  // ---- one item of one or two group records ----
+  __device__ __forceinline__ void groups(const unsigned char* rec0, bool has_b) {
+    const unsigned char* recs[2] = {rec0, has_b ? rec0 + C::kRec : rec0};
+
+    // key-min term of both groups: rows g <- group A, rows g+8 <- group B
+    float cmin[kChunks][4];
+#pragma unroll
+    for (int c = 0; c < kChunks; ++c)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) cmin[c][r] = 0.f;
+    {
+      const __half* kmA = reinterpret_cast<const __half*>(recs[0] + geo.k_min_off());
+      const __half* kmB = reinterpret_cast<const __half*>(recs[1] + geo.k_min_off());
+#pragma unroll
+      for (int s = 0; s < kKSteps; ++s) {
+        const int c0 = 16 * s + 4 * tig;
+        const uint2 x = *reinterpret_cast<const uint2*>(kmA + c0);
+        const uint2 y = *reinterpret_cast<const uint2*>(kmB + c0);
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) mma_f16(cmin[c], x.x, y.x, x.y, y.y, qb[c][s][0], qb[c][s][1]);
+      }
+    }
+    // scores in units of 2^-kCodeShift: sc[grp][c][mt][row half]
+    constexpr float kInv = 1.f / (1 << C::kCodeShift);
+    float sc[2][kChunks][2][2];
+#pragma unroll
+    for (int grp = 0; grp < 2; ++grp) {
+      const unsigned char* rec = recs[grp];
+      const __half* kscale = reinterpret_cast<const __half*>(rec + geo.k_scale_off());
+      float cacc[2][kChunks][4];
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) {
+          // a missing second group scores -inf: p = 0, the max is unchanged
+          cacc[mt][c][0] = cacc[mt][c][2] = (grp == 1 && !has_b) ? -INFINITY : cmin[c][2 * grp] * kInv;
+          cacc[mt][c][1] = cacc[mt][c][3] = 0.f;
+        }
+#pragma unroll
+      for (int w = 0; w < kLaneWordsK; ++w) {
+        uint32_t bq[kChunks][kStepsPerWord][2];
+#pragma unroll
+        for (int sl = 0; sl < kStepsPerWord; ++sl) {
+          const int s = w * kStepsPerWord + sl;
+          const uint2 ks = *reinterpret_cast<const uint2*>(kscale + 16 * s + 4 * tig);
 #pragma unroll
           for (int c = 0; c < kChunks; ++c) {
-            // hi = RN(q'' s) for even g; lo = RN(q'' s - hi) for odd g
-            bq[c][s][0] = hfma2(qq[c][s][0], ks.x, hmul2(hmul2(qq[c][s][0], ks.x), negm));
-            bq[c][s][1] = hfma2(qq[c][s][1], ks.y, hmul2(hmul2(qq[c][s][1], ks.y), negm));
+            bq[c][sl][0] = hfma2(qa[c][s][0], ks.x, hmul2(qb[c][s][0], ks.x));
+            bq[c][sl][1] = hfma2(qa[c][s][1], ks.y, hmul2(qb[c][s][1], ks.y));
           }
         }
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt) {
-          float cacc[kChunks][4];
-#pragma unroll
-          for (int c = 0; c < kChunks; ++c) {
-            // a missing second group scores -inf: p = 0, the max is unchanged
-            cacc[c][0] = cacc[c][2] = (grp == 1 && !has_b) ? -INFINITY : cmin[c][2 * grp];
-            cacc[c][1] = cacc[c][3] = 0.f;
-          }
-          const uint32_t* row0 = reinterpret_cast<const uint32_t*>(rec) +
-                                 (16 * mt + g) * geo.k_row_words() + tig * kThrWords;
-          const uint32_t* row1 = row0 + 8 * geo.k_row_words();
-          uint32_t w0[kThrWords], w1[kThrWords];
-          if constexpr (kThrWords == 4) {
-            const uint4 x0 = *reinterpret_cast<const uint4*>(row0);
-            const uint4 x1 = *reinterpret_cast<const uint4*>(row1);
-            w0[0] = x0.x; w0[1] = x0.y; w0[2] = x0.z; w0[3] = x0.w;
-            w1[0] = x1.x; w1[1] = x1.y; w1[2] = x1.z; w1[3] = x1.w;
-          } else if constexpr (kThrWords == 2) {
-            const uint2 x0 = *reinterpret_cast<const uint2*>(row0);
-            const uint2 x1 = *reinterpret_cast<const uint2*>(row1);
-            w0[0] = x0.x; w0[1] = x0.y;
-            w1[0] = x1.x; w1[1] = x1.y;
-          } else {
-            w0[0] = row0[0];
-            w1[0] = row1[0];
-          }
-#pragma unroll
-          for (int w = 0; w < kThrWords; ++w) {
-            const uint32_t h0 = w0[w] >> CW::kHiShift;
-            const uint32_t h1 = w1[w] >> CW::kHiShift;
-            constexpr int kStepsPerWord = 8 / BITS;
-#pragma unroll
-            for (int sw = 0; sw < kStepsPerWord; ++sw) {
-              const int s = w * kStepsPerWord + sw;
-              uint32_t a0, a1, a2, a3;
-              if (sw == 0) {
-                a0 = CW::template pair<0>(w0[w], h0, kc); a1 = CW::template pair<0>(w1[w], h1, kc);
-                a2 = CW::template pair<1>(w0[w], h0, kc); a3 = CW::template pair<1>(w1[w], h1, kc);
-              } else if (sw == 1) {
-                a0 = CW::template pair<2>(w0[w], h0, kc); a1 = CW::template pair<2>(w1[w], h1, kc);
-                a2 = CW::template pair<3>(w0[w], h0, kc); a3 = CW::template pair<3>(w1[w], h1, kc);
-              } else if (sw == 2) {
-                a0 = CW::template pair<4 % (16 / BITS)>(w0[w], h0, kc);
-                a1 = CW::template pair<4 % (16 / BITS)>(w1[w], h1, kc);
-                a2 = CW::template pair<5 % (16 / BITS)>(w0[w], h0, kc);
-                a3 = CW::template pair<5 % (16 / BITS)>(w1[w], h1, kc);
-              } else {
-                a0 = CW::template pair<6 % (16 / BITS)>(w0[w], h0, kc);
-                a1 = CW::template pair<6 % (16 / BITS)>(w1[w], h1, kc);
-                a2 = CW::template pair<7 % (16 / BITS)>(w0[w], h0, kc);
-                a3 = CW::template pair<7 % (16 / BITS)>(w1[w], h1, kc);
-              }
-#pragma unroll
-              for (int c = 0; c < kChunks; ++c)
-                mma_f16(cacc[c], a0, a1, a2, a3, bq[c][s][0], bq[c][s][1]);
-            }
-          }
-#pragma unroll
-          for (int c = 0; c < kChunks; ++c) {
-            sc[grp][c][mt][0] = cacc[c][0] + cacc[c][1];  // token 16mt + g, head 4c + tig
-            sc[grp][c][mt][1] = cacc[c][2] + cacc[c][3];  // token 16mt + g + 8
-          }
+          const uint32_t* row = reinterpret_cast<const uint32_t*>(rec) +
+                                (16 * mt + g) * geo.k_row_words() + tig * kLaneWordsK + w;
+          uint32_t m0, m2, n0, n2;
+          key_masks<BITS>(row[0], m0, m2);
+          key_masks<BITS>(row[8 * geo.k_row_words()], n0, n2);
+          score_steps<0>(m0, m2, n0, n2, bq, cacc[mt]);
         }
       }
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) {
+          sc[grp][c][mt][0] = cacc[mt][c][0] + cacc[mt][c][1];  // token 16mt + g, head 4c + tig
+          sc[grp][c][mt][1] = cacc[mt][c][2] + cacc[mt][c][3];  // token 16mt + g + 8
+        }
+    }
 
-      // ---- online softmax over the 64 tokens, head 4c + tig (log2 units) ----
-      float alpha[kChunks];
+    // ---- online softmax over the 64 tokens, head 4c + tig (log2 units) ----
+    float alpha[kChunks];
 #pragma unroll
-      for (int c = 0; c < kChunks; ++c) {
-        // max of the raw MMA scores (ch > 0 keeps the order), then log2 units
-        float mx = fmaxf(fmaxf(fmaxf(sc[0][c][0][0], sc[0][c][0][1]),
-                               fmaxf(sc[0][c][1][0], sc[0][c][1][1])),
-                         fmaxf(fmaxf(sc[1][c][0][0], sc[1][c][0][1]),
-                               fmaxf(sc[1][c][1][0], sc[1][c][1][1])));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-        const float m_new = fmaxf(m_run[c], mx * ch[c]);
-        alpha[c] = fast_exp2(m_run[c] - m_new);
-        m_run[c] = m_new;
-        float sum = 0.f;
-        __half* prow = p_s + (4 * c + tig) * kPRow;
+    for (int c = 0; c < kChunks; ++c) {
+      // max of the raw MMA scores (ch > 0 keeps the order), then log2 units
+      float mx = fmaxf(fmaxf(fmaxf(sc[0][c][0][0], sc[0][c][0][1]),
+                             fmaxf(sc[0][c][1][0], sc[0][c][1][1])),
+                       fmaxf(fmaxf(sc[1][c][0][0], sc[1][c][0][1]),
+                             fmaxf(sc[1][c][1][0], sc[1][c][1][1])));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      const float m_new = fmaxf(m_run[c], mx * ch[c]);
+      alpha[c] = fast_exp2(m_run[c] - m_new);
+      m_run[c] = m_new;
+      float sum = 0.f;
 #pragma unroll
-        for (int grp = 0; grp < 2; ++grp)
+      for (int grp = 0; grp < 2; ++grp)
 #pragma unroll
-          for (int mt = 0; mt < 2; ++mt)
+        for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-            for (int hr = 0; hr < 2; ++hr) {
-              const float pv = fast_exp2(fmaf(sc[grp][c][mt][hr], ch[c], -m_new));
-              sum += pv;
-              prow[grp * kGroup + 16 * mt + 8 * hr + g] = __float2half_rn(pv);
-            }
-        l_run[c] = l_run[c] * alpha[c] + sum;
-      }
-      __syncwarp();
-
-      // ---- rescale the P.V accumulators (columns = heads 2tig, 2tig+1) ----
-      bool same = true;
-#pragma unroll
-      for (int c = 0; c < kChunks; ++c) same = same && alpha[c] == 1.f;
-      if (!__all_sync(0xffffffffu, same)) {
-        float al[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int h = 2 * tig + e;
-          const int src = 4 * g + (h & 3);
-          float v0 = __shfl_sync(0xffffffffu, alpha[0], src);
-          if constexpr (kChunks == 2) {
-            const float v1 = __shfl_sync(0xffffffffu, alpha[kChunks - 1], src);
-            v0 = h >= 4 ? v1 : v0;
+          for (int hr = 0; hr < 2; ++hr) {
+            const float pv = fast_exp2(fmaf(sc[grp][c][mt][hr], ch[c], -m_new));
+            sum += pv;
+            store_p(c, grp * kGroup + 16 * mt + 8 * hr + g, pv);
           }
-          al[e] = v0;
-        }
-#pragma unroll
-        for (int mt = 0; mt < kMTiles; ++mt) {
-          acc[mt][0] *= al[0];
-          acc[mt][1] *= al[1];
-          acc[mt][2] *= al[0];
-          acc[mt][3] *= al[1];
-        }
-        vmacc[0] *= al[0];
-        vmacc[1] *= al[1];
-        vmacc[2] *= al[0];
-        vmacc[3] *= al[1];
-      }
+      l_run[c] = l_run[c] * alpha[c] + sum;
+    }
+    __syncwarp();
+    rescale(alpha);
 
-      // ---- P.V of both groups ----
+    // ---- P.V of both groups ----
 #pragma unroll
-      for (int grp = 0; grp < 2; ++grp) {
-        const unsigned char* rec = recs[grp];
-        const __half* vscale = reinterpret_cast<const __half*>(rec + geo.v_scale_off());
-        const __half* vmin = reinterpret_cast<const __half*>(rec + geo.v_min_off());
-        // B: p of head g, tokens (16kk + 8hf + 2tig, +1)
-        uint32_t pb[2][2];
+    for (int grp = 0; grp < 2; ++grp) {
+      const unsigned char* rec = recs[grp];
+      const __half* vscale = reinterpret_cast<const __half*>(rec + geo.v_scale_off());
+      const __half* vmin = reinterpret_cast<const __half*>(rec + geo.v_min_off());
+      // p of tokens (16kk + 8hf + 2tig, +1) for this lane's B column
+      uint32_t pa[2][2], px[2][2];
+#pragma unroll
+      for (int kk = 0; kk < 2; ++kk)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const uint32_t col = (uint32_t)(grp * kGroup + 16 * kk + 8 * hf + 2 * tig) * 2;
+          pa[kk][hf] = lds32(p_tile + rowA + col);
+          px[kk][hf] = lds32(p_tile + rowX + col);
+        }
+      // this lane's V-code words
+      const uint32_t* vw = reinterpret_cast<const uint32_t*>(rec + geo.v_codes_off()) + lane * 4;
+      uint32_t vwords[kVWords];
+#pragma unroll
+      for (int q4 = 0; q4 < kVWords / 4; ++q4) {
+        const uint4 x = *reinterpret_cast<const uint4*>(vw + q4 * 128);
+        vwords[4 * q4] = x.x;
+        vwords[4 * q4 + 1] = x.y;
+        vwords[4 * q4 + 2] = x.z;
+        vwords[4 * q4 + 3] = x.w;
+      }
+      // value-min term: rows g -> block g % kBlocks
+      {
+        const uint4 vm = *reinterpret_cast<const uint4*>(vmin + 32 * (g % kBlocks) + 8 * tig);
+        if constexpr (C::kLoCols) {
+          // hi columns: p_hi; lo columns: -p_lo
+          mma_f16(vmacc, vm.x, vm.x, vm.y, vm.y, and_or(pa[0][0], maskHi, px[0][0]),
+                  and_or(pa[0][1], maskHi, px[0][1]));
+          mma_f16(vmacc, vm.z, vm.z, vm.w, vm.w, and_or(pa[1][0], maskHi, px[1][0]),
+                  and_or(pa[1][1], maskHi, px[1][1]));
+        } else {
+          mma_f16(vmacc, vm.x, vm.x, vm.y, vm.y, pa[0][0], pa[0][1]);
+          mma_f16(vmacc, vm.z, vm.z, vm.w, vm.w, pa[1][0], pa[1][1]);
+          mma_f16(vmacc, vm.x, vm.x, vm.y, vm.y, px[0][0], px[0][1]);
+          mma_f16(vmacc, vm.z, vm.z, vm.w, vm.w, px[1][0], px[1][1]);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kBlocks; ++j) {
+        const uint4 vs4 = *reinterpret_cast<const uint4*>(vscale + 32 * j + 8 * tig);
+        const uint32_t vs[2][2] = {{vs4.x, vs4.y}, {vs4.z, vs4.w}};
+        uint32_t pt[2][2], pl[2][2];
 #pragma unroll
         for (int kk = 0; kk < 2; ++kk)
 #pragma unroll
-          for (int hf = 0; hf < 2; ++hf)
-            pb[kk][hf] = *reinterpret_cast<const uint32_t*>(p_s + g * kPRow + grp * kGroup +
-                                                            16 * kk + 8 * hf + 2 * tig);
-        // value-min term, deferred: rows g -> block g % kBlocks
-        {
-          const uint4 vm = *reinterpret_cast<const uint4*>(vmin + 32 * (g % kBlocks) + 8 * tig);
-          mma_f16(vmacc, vm.x, vm.x, vm.y, vm.y, pb[0][0], pb[0][1]);
-          mma_f16(vmacc, vm.z, vm.z, vm.w, vm.w, pb[1][0], pb[1][1]);
-        }
-        // this thread's V-code words: (4g + tig) * kVWords ... + kVWords - 1
-        const uint32_t* vw = reinterpret_cast<const uint32_t*>(rec + geo.v_codes_off()) +
-                             (4 * g + tig) * kVWords;
-        uint32_t vwords[kVWords];
-#pragma unroll
-        for (int q4 = 0; q4 < kVWords / 4; ++q4) {
-          const uint4 x = *reinterpret_cast<const uint4*>(vw + 4 * q4);
-          vwords[4 * q4] = x.x; vwords[4 * q4 + 1] = x.y;
-          vwords[4 * q4 + 2] = x.z; vwords[4 * q4 + 3] = x.w;
-        }
-#pragma unroll
-        for (int j = 0; j < kBlocks; ++j) {
-          const uint4 vs = *reinterpret_cast<const uint4*>(vscale + 32 * j + 8 * tig);
-          const uint32_t pt00 = hmul2(pb[0][0], vs.x), pt01 = hmul2(pb[0][1], vs.y);
-          const uint32_t pt10 = hmul2(pb[1][0], vs.z), pt11 = hmul2(pb[1][1], vs.w);
-#pragma unroll
-          for (int mi = 0; mi < 2; ++mi) {
-            const int mt = 2 * j + mi;
-            if constexpr (BITS == 2) {
-              const uint32_t x = vwords[mt], xh = x >> CW::kHiShift;
-              // pairs idx = 4kk + 2hf + r: a0 (r0,hf0), a1 (r1,hf0), a2 (r0,hf1), a3 (r1,hf1)
-              mma_f16(acc[mt], CW::template pair<0>(x, xh, kc), CW::template pair<1>(x, xh, kc),
-                      CW::template pair<2>(x, xh, kc), CW::template pair<3>(x, xh, kc), pt00, pt01);
-              mma_f16(acc[mt], CW::template pair<4>(x, xh, kc), CW::template pair<5>(x, xh, kc),
-                      CW::template pair<6>(x, xh, kc), CW::template pair<7>(x, xh, kc), pt10, pt11);
+          for (int hf = 0; hf < 2; ++hf) {
+            if constexpr (C::kLoCols) {
+              // hi columns: RN(p_hi vs); lo columns: -RN(p_lo vs + (p_hi vs - hi))
+              const uint32_t y = and_xor(pa[kk][hf], maskY, signY);
+              pt[kk][hf] = hfma2(px[kk][hf], vs[kk][hf],
+                                 hfma2(y, vs[kk][hf], hmul2(pa[kk][hf], vs[kk][hf])));
             } else {
-              const uint32_t x0 = vwords[2 * mt], x0h = x0 >> CW::kHiShift;
-              const uint32_t x1 = vwords[2 * mt + 1], x1h = x1 >> CW::kHiShift;
-              mma_f16(acc[mt], CW::template pair<0>(x0, x0h, kc), CW::template pair<1>(x0, x0h, kc),
-                      CW::template pair<2>(x0, x0h, kc), CW::template pair<3>(x0, x0h, kc), pt00, pt01);
-              mma_f16(acc[mt], CW::template pair<0>(x1, x1h, kc), CW::template pair<1>(x1, x1h, kc),
-                      CW::template pair<2>(x1, x1h, kc), CW::template pair<3>(x1, x1h, kc), pt10, pt11);
+              const uint32_t nhi = hmul2(pa[kk][hf] ^ 0x80008000u, vs[kk][hf]);
+              pl[kk][hf] = hfma2(px[kk][hf], vs[kk][hf], hfma2(pa[kk][hf], vs[kk][hf], nhi));
+              pt[kk][hf] = nhi ^ 0x80008000u;
             }
           }
-        }
-      }
-
-      // release both stages and refill them with groups i + kStages, i + 1 + kStages
-      __syncwarp();
-      if (lane == 0) {
-        fence_proxy_async();
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int k = i + e + kStages;
-          if (i + e < n_mine && k < n_mine) {
-            const int st = (i + e) % kStages;
-            mbar_expect_tx(&bars[st], P::kRec);
-            bulk_load(stage0 + st * P::kRec,
-                      seq_rec + (long)(first + warp + k * kWarps) * P::kRec, P::kRec, &bars[st]);
+        for (int mi = 0; mi < 2; ++mi) {
+          const int mt = 2 * j + mi;
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk) {
+            uint32_t va[4];
+            value_operands<BITS>(BITS == 2 ? vwords[mt] : vwords[2 * mt + kk], kk, va);
+            mma_f16(acc[mt], va[0], va[1], va[2], va[3], pt[kk][0], pt[kk][1]);
+            if constexpr (!C::kLoCols)
+              mma_f16(acc[mt], va[0], va[1], va[2], va[3], pl[kk][0], pl[kk][1]);
           }
         }
       }
     }
+  }
 
-    if (timed_out && lane == 0) {
-      // record the failure, then give the copies already issued (local groups
-      // i_stop .. i_stop + kStages - 1) a bounded chance to land before this
-      // CTA's shared memory is reused
-      atomicOr(args.status, kStatusWaitTimeout);
-      for (int k = i_stop; k < n_mine && k < i_stop + kStages; ++k)
-        (void)mbar_wait_bounded(&bars[k % kStages], (uint32_t)(k / kStages) & 1u);
+  // ---- one residual item: n (1..8) ring tokens, K rows then V rows (padded) ----
+  __device__ __forceinline__ void residual(unsigned char* base, int n) {
+    const uint32_t kbase = smem_addr(base), vbase = smem_addr(base + C::kRec);
+    if (n < kResTok) {  // rows past the last token: zero V (0 * stale data must stay 0)
+      constexpr int kVec = 2 * D / 16;
+      for (int i = lane; i < (kResTok - n) * kVec; i += 32) {
+        const int t = n + i / kVec, c = i % kVec;
+        *reinterpret_cast<uint4*>(base + C::kRec + t * C::kResRow + 16 * c) =
+            make_uint4(0u, 0u, 0u, 0u);
+      }
+      __syncwarp();
     }
-    // row sums over the 8 token lanes of each head
+    // scores: rows = tokens (0..7), columns 2h = head 4c + h (q in bf16), 2h+1 = 0
+    float sacc[kChunks][4];
+#pragma unroll
+    for (int c = 0; c < kChunks; ++c)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) sacc[c][r] = 0.f;
+    const int mrow = lane & 7, mat = lane >> 3;
+#pragma unroll
+    for (int s = 0; s < kKSteps; s += 2) {
+      uint32_t kf[4];  // (s: a0, a2), (s+1: a0, a2)
+      ldsm_x4(kf, kbase + mrow * C::kResRow + (16 * (s + mat / 2) + 8 * (mat % 2)) * 2);
+#pragma unroll
+      for (int c = 0; c < kChunks; ++c) {
+        const int h = 4 * c + g / 2;
+        const bool live = (g % 2) == 0 && h < HPK;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int ch0 = 16 * (s + u) + 2 * tig;
+          const uint32_t b0 = live ? *reinterpret_cast<const uint32_t*>(q_pair + h * D + ch0) : 0u;
+          const uint32_t b1 =
+              live ? *reinterpret_cast<const uint32_t*>(q_pair + h * D + ch0 + 8) : 0u;
+          mma_bf16(sacc[c], kf[2 * u], 0u, kf[2 * u + 1], 0u, b0, b1);
+        }
+      }
+    }
+    // online softmax: one token (g) per lane, head 4c + tig
+    float alpha[kChunks];
+    constexpr float kInv = 1.f / (1 << C::kCodeShift);
 #pragma unroll
     for (int c = 0; c < kChunks; ++c) {
-      l_run[c] += __shfl_xor_sync(0xffffffffu, l_run[c], 4);
-      l_run[c] += __shfl_xor_sync(0xffffffffu, l_run[c], 8);
-      l_run[c] += __shfl_xor_sync(0xffffffffu, l_run[c], 16);
-    }
-    // add the deferred value-min term: block j of head 2tig+e sits in lane 4j + tig
-#pragma unroll
-    for (int j = 0; j < kBlocks; ++j) {
-      const float v0 = __shfl_sync(0xffffffffu, vmacc[0], 4 * j + tig);
-      const float v1 = __shfl_sync(0xffffffffu, vmacc[1], 4 * j + tig);
-#pragma unroll
-      for (int mi = 0; mi < 2; ++mi) {
-        acc[2 * j + mi][0] += v0;
-        acc[2 * j + mi][2] += v0;
-        acc[2 * j + mi][1] += v1;
-        acc[2 * j + mi][3] += v1;
-      }
-    }
-    __syncthreads();  // every warp is done with its stages: the merge area may alias them
-#pragma unroll
-    for (int c = 0; c < kChunks; ++c) {
-      const int hh = 4 * c + tig;
-      if (hh < HPK && g == 0) {
-        wm[warp * 8 + hh] = n_mine > 0 ? m_run[c] : -INFINITY;
-        wl[warp * 8 + hh] = n_mine > 0 ? l_run[c] : 0.f;
-      }
-    }
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int hh = 2 * tig + e;
-      if (hh < HPK) {
-#pragma unroll
-        for (int mt = 0; mt < kMTiles; ++mt) {
-          merge_acc[(warp * HPK + hh) * D + 16 * mt + g] = acc[mt][e];
-          merge_acc[(warp * HPK + hh) * D + 16 * mt + g + 8] = acc[mt][e + 2];
-        }
-      }
-    }
-  } else {
-    // ============ residual CTA: one chunk of <= 32 bf16 ring tokens, CUDA cores ============
-    // The chunk's K and V rows are staged in shared memory (one coalesced pass;
-    // a chunk starts at a multiple of 32 tokens, so its ring slots are
-    // contiguous), then scores, the chunk softmax and P.V read shared memory.
-    // This CTA writes its partial directly and returns.
-    allow_successor();
-    const int chunk = split - splits_g;
-    const int t0 = NG * kGroup + chunk * kGroup;
-    const int n = min(kGroup, S - t0);
-    const int slot0 = t0 % kRingSlots;
-    __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(smem);  // [32][D]
-    __nv_bfloat16* vc = kc + kGroup * D;                          // [32][D]
-    float* s_res = reinterpret_cast<float*>(vc + kGroup * D);     // [HPK][32]
-    static_assert(2 * kGroup * D * 2 + HPK * kGroup * 4 <= P::kStageBytes,
-                  "residual chunk must fit in the stage area");
-    {
-      // every load of the chunk is issued before the first store: one round trip
-      const uint4* gk = reinterpret_cast<const uint4*>(args.ring_k + (seq * kRingSlots + slot0) * D);
-      const uint4* gv = reinterpret_cast<const uint4*>(args.ring_v + (seq * kRingSlots + slot0) * D);
-      const int n16 = n * D * 2 / 16;
-      constexpr int kPer = (kGroup * D * 2 / 16 + kThreads - 1) / kThreads;
-      uint4 rk[kPer], rv[kPer];
-#pragma unroll
-      for (int k = 0; k < kPer; ++k) {
-        const int i = threadIdx.x + k * kThreads;
-        if (i < n16) {
-          rk[k] = gk[i];
-          rv[k] = gv[i];
-        }
-      }
-#pragma unroll
-      for (int k = 0; k < kPer; ++k) {
-        const int i = threadIdx.x + k * kThreads;
-        if (i < n16) {
-          reinterpret_cast<uint4*>(kc)[i] = rk[k];
-          reinterpret_cast<uint4*>(vc)[i] = rv[k];
-        }
-      }
-    }
-    __syncthreads();
-    // scores: one (token, head) pair per thread step; each thread walks the
-    // channel pairs starting at an offset set by its token (spreads the banks)
-    for (int pidx = threadIdx.x; pidx < kGroup * HPK; pidx += kThreads) {
-      const int t = pidx / HPK, hh = pidx % HPK;
-      float sum = -INFINITY;
-      if (t < n) {
-        sum = 0.f;
-        const __nv_bfloat162* kr = reinterpret_cast<const __nv_bfloat162*>(kc + t * D);
-        const float2* qr = reinterpret_cast<const float2*>(q_s + hh * D);
-#pragma unroll 8
-        for (int w = 0; w < D / 2; ++w) {
-          const int ww = (w + t) & (D / 2 - 1);
-          const float2 kf = __bfloat1622float2(kr[ww]);
-          const float2 qf = qr[ww];
-          sum = fmaf(kf.x, qf.x, fmaf(kf.y, qf.y, sum));
-        }
-        sum *= qscale;
-      }
-      s_res[hh * kGroup + t] = sum;
-    }
-    __syncthreads();
-    // chunk softmax per head: warp w takes heads w, w + 4, ...
-    for (int hh = warp; hh < HPK; hh += kWarps) {
-      const float x = s_res[hh * kGroup + lane];
+      const float x = g < n ? sacc[c][0] * qscale : -INFINITY;
       float mx = x;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      const float pv = exp2f(x - mx);
-      float l = pv;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-      s_res[hh * kGroup + lane] = pv;
-      if (lane == 0) {
-        wm[hh] = mx;
-        wl[hh] = l;
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      const float m_new = fmaxf(m_run[c], mx);
+      alpha[c] = fast_exp2(m_run[c] - m_new);
+      m_run[c] = m_new;
+      const float pv = fast_exp2(x - m_new);
+      l_run[c] = l_run[c] * alpha[c] + pv;
+      // p / 2^shift as bf16 hi (tile columns 0..7) + lo (8..15): the accumulators
+      // hold the group terms in units of 2^-shift as well
+      const int h = 4 * c + tig;
+      if (h < HPK) {
+        const float ps = pv * kInv;
+        const __nv_bfloat16 hi = __float2bfloat16_rn(ps);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(ps - __bfloat162float(hi));
+        __nv_bfloat16* row = reinterpret_cast<__nv_bfloat16*>(p_tile) + h * kPRow;
+        row[g] = hi;
+        row[8 + g] = lo;
       }
     }
-    __syncthreads();
-    const int splits_total = splits_g + n_res;
-    const long part0 = ((long)b * Hq + kvh * HPK) * splits_total + split;
-    for (int i = threadIdx.x; i < HPK * D; i += kThreads) {
-      const int hh = i / D, d = i % D;
-      float o = 0.f;
-      for (int t = 0; t < n; ++t)
-        o = fmaf(s_res[hh * kGroup + t], __bfloat162float(vc[t * D + d]), o);
-      args.ws_acc[(part0 + (long)hh * splits_total) * D + d] = o;
+    __syncwarp();
+    rescale(alpha);
+    // P.V: A = V^T (channels x tokens) from ldmatrix.trans; k = 0..7 with p_hi,
+    // k = 8..15 the same tokens with p_lo
+    const uint32_t b0 = lds32(p_tile + rowR + 2 * tig * 2);
+    const uint32_t b1 = lds32(p_tile + rowR + (8 + 2 * tig) * 2);
+#pragma unroll
+    for (int mt = 0; mt < kMTiles; mt += 2) {
+      uint32_t vf[4];  // (mt: a0, a1), (mt+1: a0, a1)
+      ldsm_x4_trans(vf, vbase + mrow * C::kResRow + (16 * (mt + mat / 2) + 8 * (mat % 2)) * 2);
+      mma_bf16(acc[mt], vf[0], vf[1], vf[0], vf[1], b0, b1);
+      mma_bf16(acc[mt + 1], vf[2], vf[3], vf[2], vf[3], b0, b1);
     }
-    if (threadIdx.x < HPK) {
-      const int hh = threadIdx.x;
-      args.ws_ml[2 * (part0 + (long)hh * splits_total)] = wm[hh];
-      args.ws_ml[2 * (part0 + (long)hh * splits_total) + 1] = wl[hh];
-    }
+  }
+};
+
+template <int D, int BITS, int HPK>
+__global__ void __launch_bounds__(Cfg<D, BITS, HPK>::kThreads, 1)
+decode_kernel(DecodeArgs args, Split sp) {
+  using C = Cfg<D, BITS, HPK>;
+  using W = Warp<D, BITS, HPK>;
+  using Slot = PairSlot<D, HPK>;
+  static_assert(sizeof(Slot) <= C::kSlotBytes, "pair slot size");
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int cta = blockIdx.x;
+
+  const int it_begin = cta_first_item(sp, cta), it_end = cta_first_item(sp, cta + 1);
+  const int p_first = it_begin / sp.ipp, p_last = (it_end - 1) / sp.ipp;
+  const int n_pairs = p_last - p_first + 1;
+  unsigned char* wbase = smem + warp * C::kWarpBytes;
+  Slot* slots = reinterpret_cast<Slot*>(smem + C::kOffSlots);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffFixed) + 2 * warp;
+  int* s_ctr = reinterpret_cast<int*>(smem + C::kOffFixed + 8 * 2 * C::kNW);
+  int* s_flag = s_ctr + 1;
+  if (it_end <= it_begin || n_pairs > C::kSlots) {  // the host's split rules exclude both
+    if (threadIdx.x == 0) atomicOr(args.status, kStatusBadSplit);
     return;
   }
 
-  allow_successor();
-  // ===================== merge the warps, write this CTA's partial =====================
-  __syncthreads();
-  const int splits_total = splits_g + n_res;
-  const long part0 = ((long)b * Hq + kvh * HPK) * splits_total + split;
-  for (int i = threadIdx.x; i < HPK * D; i += kThreads) {
-    const int hh = i / D, d = i % D;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, wm[w * 8 + hh]);
-    float o = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      const float mw = wm[w * 8 + hh];
-      if (mw != -INFINITY) o += exp2f(mw - M) * merge_acc[(w * HPK + hh) * D + d];
+  // ---- set-up: p tiles, mbarriers, pair slots, the claim counter ----
+  {
+    uint32_t* pt = reinterpret_cast<uint32_t*>(wbase + 2 * C::kItemBytes);
+    for (int i = lane; i < C::kPRows * kPRow / 2; i += 32) pt[i] = 0u;
+    if (lane == 0) {
+      mbar_init(&bars[0], 1);
+      mbar_init(&bars[1], 1);
+      fence_mbar_init();
     }
-    args.ws_acc[(part0 + (long)hh * splits_total) * D + d] = o;
+    for (int k = warp; k < n_pairs; k += C::kNW) {
+      Slot& sl = slots[k];
+      if (lane < 8) {
+        sl.m[lane] = -INFINITY;
+        sl.l[lane] = 0.f;
+      }
+      if (lane == 0) sl.lock = 0;
+      for (int i = lane; i < HPK * D; i += 32) (&sl.acc[0][0])[i] = 0.f;
+    }
+    if (threadIdx.x == 0) *s_ctr = it_begin;
   }
-  if (threadIdx.x < HPK) {
-    const int hh = threadIdx.x;
+  wait_for_predecessor();  // q, the records and the rings may come from the previous kernel
+  for (int k = warp; k < n_pairs; k += C::kNW) {
+    const int pair = p_first + k;
+    const int b = pair / args.Hkv, kvh = pair % args.Hkv;
+    const uint4* src =
+        reinterpret_cast<const uint4*>(args.q + ((long)b * args.Hq + (long)kvh * HPK) * D);
+    uint4* dst = reinterpret_cast<uint4*>(&slots[k].q[0][0]);
+    for (int i = lane; i < HPK * D / 8; i += 32) dst[i] = src[i];
+  }
+  __syncthreads();
+
+  const float qscale = (args.sm_scale > 0.f ? args.sm_scale : rsqrtf((float)D)) * kLog2e;
+  W w(args, lane, qscale);
+  w.p_tile = wbase + 2 * C::kItemBytes;
+  {
+    const int hcol = w.g & 3;
+    const bool lo_lane = C::kLoCols && w.g >= 4;
+    constexpr int kRowBytes = kPRow * 2;
+    if constexpr (C::kLoCols) {
+      w.rowA = (hcol < HPK ? hcol : C::kZeroRow) * kRowBytes;
+      w.rowX = (lo_lane && hcol < HPK ? HPK + hcol : C::kZeroRow) * kRowBytes;
+      w.rowR = (!lo_lane && hcol < HPK ? hcol : C::kZeroRow) * kRowBytes;
+    } else {
+      w.rowA = w.g * kRowBytes;
+      w.rowX = (HPK + w.g) * kRowBytes;
+      w.rowR = w.g * kRowBytes;
+    }
+    w.maskY = lo_lane ? 0xffffffffu : 0u;
+    w.signY = lo_lane ? 0x80008000u : 0u;
+    w.maskHi = lo_lane ? 0u : 0xffffffffu;
+  }
+  w.reset();
+
+  const int NG = sp.NG, S = args.S;
+  const long rec_stride = C::kRec;
+  // claims the next item (warp-uniform result; -1 when the CTA's range is done)
+  auto claim = [&]() -> int {
+    int it = 0;
+    if (lane == 0) it = atomicAdd(s_ctr, 1);
+    it = __shfl_sync(0xffffffffu, it, 0);
+    return it < it_end ? it : -1;
+  };
+  // lane 0 starts the copies of item `it` into item slot k
+  auto issue = [&](int it, int k) {
+    if (lane != 0 || it < 0) return;
+    unsigned char* dst = wbase + k * C::kItemBytes;
+    const int pair = it / sp.ipp, kk = it % sp.ipp;
+    if (kk < sp.n2 + sp.n1) {
+      const int g0 = 2 * kk;
+      const uint32_t bytes = (kk < sp.n2 ? 2 : 1) * C::kRec;
+      mbar_expect_tx(&bars[k], bytes);
+      bulk_load(dst, args.records + ((long)pair * args.ngcap + g0) * rec_stride, bytes, &bars[k]);
+    } else {
+      const int t0 = NG * kGroup + kResTok * (kk - sp.n2 - sp.n1);
+      const int n = min(kResTok, S - t0);
+      const long row0 = (long)pair * kRingSlots + t0 % kRingSlots;
+      mbar_expect_tx(&bars[k], 2u * n * D * 2);
+      for (int t = 0; t < n; ++t) {
+        bulk_load(dst + t * C::kResRow, args.ring_k + (row0 + t) * D, D * 2, &bars[k]);
+        bulk_load(dst + C::kRec + t * C::kResRow, args.ring_v + (row0 + t) * D, D * 2, &bars[k]);
+      }
+    }
+  };
+
+  int itm[2];
+  itm[0] = claim();
+  issue(itm[0], 0);
+  itm[1] = claim();
+  issue(itm[1], 1);
+  int cur_pair = -1;
+  bool timed_out = false;
+  int i_stop = 0;
+
+  // merges this warp's state for `pair` into the CTA's slot
+  auto flush = [&](int pair) {
+    Slot& sl = slots[pair - p_first];
+    float lw[C::kChunks];
+#pragma unroll
+    for (int c = 0; c < C::kChunks; ++c) {
+      float l = w.l_run[c];
+      l += __shfl_xor_sync(0xffffffffu, l, 4);
+      l += __shfl_xor_sync(0xffffffffu, l, 8);
+      l += __shfl_xor_sync(0xffffffffu, l, 16);
+      lw[c] = l;
+    }
+    // final accumulators: (hi - lo') for <= 4 heads, times 2^shift, plus the value-min term
+    float F[W::kMTiles][4];
+    float vm[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) vm[r] = w.vmacc[r];
+#pragma unroll
+    for (int mt = 0; mt < W::kMTiles; ++mt)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) F[mt][r] = w.acc[mt][r];
+    if constexpr (C::kLoCols) {
+#pragma unroll
+      for (int mt = 0; mt < W::kMTiles; ++mt)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) F[mt][r] -= __shfl_xor_sync(0xffffffffu, F[mt][r], 2);
+#pragma unroll
+      for (int r = 0; r < 4; ++r) vm[r] -= __shfl_xor_sync(0xffffffffu, vm[r], 2);
+    }
+#pragma unroll
+    for (int mt = 0; mt < W::kMTiles; ++mt)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) F[mt][r] *= (float)(1 << C::kCodeShift);
+    // value-min term of block j, columns 2tig + e, sits in lane 4j + tig (rows g = j)
+#pragma unroll
+    for (int j = 0; j < W::kBlocks; ++j) {
+      const float v0 = __shfl_sync(0xffffffffu, vm[0], 4 * j + w.tig);
+      const float v1 = __shfl_sync(0xffffffffu, vm[1], 4 * j + w.tig);
+#pragma unroll
+      for (int mi = 0; mi < 2; ++mi) {
+        F[2 * j + mi][0] += v0;
+        F[2 * j + mi][2] += v0;
+        F[2 * j + mi][1] += v1;
+        F[2 * j + mi][3] += v1;
+      }
+    }
+    float Mw[2], Lw[2];
+    {
+      float mh[2], lh[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int h = 2 * w.tig + e;  // head of accumulator column 2tig + e (hi lanes)
+        const int src = (lane & ~3) | (h & 3);
+        float m0 = __shfl_sync(0xffffffffu, w.m_run[0], src);
+        float l0 = __shfl_sync(0xffffffffu, lw[0], src);
+        if constexpr (C::kChunks == 2) {
+          const float m1 = __shfl_sync(0xffffffffu, w.m_run[C::kChunks - 1], src);
+          const float l1 = __shfl_sync(0xffffffffu, lw[C::kChunks - 1], src);
+          m0 = h >= 4 ? m1 : m0;
+          l0 = h >= 4 ? l1 : l0;
+        }
+        mh[e] = m0;
+        lh[e] = l0;
+      }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        Mw[e] = mh[e];
+        Lw[e] = lh[e];
+      }
+    }
+    // lock the slot (bounded)
+    bool locked = true;
+    if (lane == 0) {
+      int spins = 0;
+      while (atomicCAS(&sl.lock, 0, 1) != 0) {
+        if (++spins > kLockSpinLimit) {
+          locked = false;
+          atomicOr(args.status, kStatusLockTimeout);
+          break;
+        }
+        __nanosleep(64);
+      }
+    }
+    locked = __shfl_sync(0xffffffffu, locked, 0);
+    if (!locked) return;
+    __threadfence_block();
+    const bool valid_lane = C::kLoCols ? w.tig < 2 : true;
+    float newM[2], newL[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int h = 2 * w.tig + e;
+      const bool valid = valid_lane && h < HPK;
+      const float Ms = sl.m[h & 7], Ls = sl.l[h & 7];
+      const float M = fmaxf(Ms, Mw[e]);
+      const float fs = Ms == -INFINITY ? 0.f : exp2f(Ms - M);
+      const float fw = Mw[e] == -INFINITY ? 0.f : exp2f(Mw[e] - M);
+      newM[e] = M;
+      newL[e] = Ls * fs + Lw[e] * fw;
+      if (valid) {
+        float* ah = sl.acc[h < HPK ? h : 0];
+#pragma unroll
+        for (int mt = 0; mt < W::kMTiles; ++mt) {
+          ah[16 * mt + w.g] = ah[16 * mt + w.g] * fs + F[mt][e] * fw;
+          ah[16 * mt + w.g + 8] = ah[16 * mt + w.g + 8] * fs + F[mt][e + 2] * fw;
+        }
+      }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int h = 2 * w.tig + e;
+      if (valid_lane && h < HPK && w.g == 0) {
+        sl.m[h] = newM[e];
+        sl.l[h] = newL[e];
+      }
+    }
+    __threadfence_block();
+    __syncwarp();
+    if (lane == 0) atomicExch(&sl.lock, 0);
+  };
+
+  for (int i = 0;; ++i) {
+    const int k = i & 1;
+    const int it = itm[k];
+    if (it < 0) break;
+    const bool arrived = mbar_wait_bounded(&bars[k], (uint32_t)(i >> 1) & 1u);
+    if (!__all_sync(0xffffffffu, arrived)) {
+      timed_out = true;
+      i_stop = i;
+      break;
+    }
+    const int pair = it / sp.ipp, kk = it % sp.ipp;
+    if (pair != cur_pair) {
+      if (cur_pair >= 0) {
+        flush(cur_pair);
+        w.reset();
+      }
+      w.load_pair(&slots[pair - p_first].q[0][0]);
+      cur_pair = pair;
+    }
+    unsigned char* base = wbase + k * C::kItemBytes;
+    if (kk < sp.n2 + sp.n1) {
+      w.groups(base, kk < sp.n2);
+    } else {
+      const int t0 = NG * kGroup + kResTok * (kk - sp.n2 - sp.n1);
+      w.residual(base, min(kResTok, S - t0));
+    }
+    // release the item slot, claim the next item and start its copies
+    __syncwarp();
+    if (lane == 0) fence_proxy_async();
+    itm[k] = claim();
+    issue(itm[k], k);
+  }
+  if (timed_out) {
+    // record the failure, then give the copies still in flight a bounded chance
+    // to land before this CTA's shared memory is released
+    if (lane == 0) {
+      atomicOr(args.status, kStatusWaitTimeout);
+      for (int j = i_stop; j < i_stop + 2; ++j)
+        if (itm[j & 1] >= 0) (void)mbar_wait_bounded(&bars[j & 1], (uint32_t)(j >> 1) & 1u);
+    }
+    __syncwarp();
+  }
+  if (cur_pair >= 0) flush(cur_pair);
+  __syncthreads();
+  allow_successor();
+
+  // ---- outputs: whole pairs directly, shared pairs through partials and tickets ----
+  constexpr int kPart = HPK * (D + 2);  // floats of one partial: m[HPK], l[HPK], acc[HPK][D]
+  for (int k = warp; k < n_pairs; k += C::kNW) {
+    const int pair = p_first + k;
+    const Slot& sl = slots[k];
+    const int fc = cta_of_item(sp, pair * sp.ipp), lc = cta_of_item(sp, pair * sp.ipp + sp.ipp - 1);
+    const int b = pair / args.Hkv, kvh = pair % args.Hkv;
+    float* out = args.out + ((long)b * args.Hq + (long)kvh * HPK) * D;
+    if (fc == lc) {
+      for (int i = lane; i < HPK * D; i += 32) out[i] = sl.acc[i / D][i % D] / sl.l[i / D];
+      continue;
+    }
+    const int side = pair == p_first ? 0 : 1;
+    if (cta >= args.max_ctas) {  // the host sizes the partials for every grid it launches
+      if (lane == 0) atomicOr(args.status, kStatusBadSplit);
+      continue;
+    }
+    float* part = args.partials + ((long)cta * 2 + side) * kPart;
+    if (lane < HPK) {
+      part[lane] = sl.m[lane];
+      part[HPK + lane] = sl.l[lane];
+    }
+    for (int i = lane; i < HPK * D; i += 32) part[2 * HPK + i] = sl.acc[i / D][i % D];
+    __threadfence();
+    __syncwarp();
+    int prev = 0;
+    if (lane == 0) prev = atomicAdd(&args.tickets[pair], 1);
+    prev = __shfl_sync(0xffffffffu, prev, 0);
+    if (prev != lc - fc) continue;
+    // the last CTA of this pair: merge the partials of CTAs fc..lc
+    __threadfence();
     float M = -INFINITY, L = 0.f;
-    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, wm[w * 8 + hh]);
-    for (int w = 0; w < kWarps; ++w)
-      if (wm[w * 8 + hh] != -INFINITY) L += wl[w * 8 + hh] * exp2f(wm[w * 8 + hh] - M);
-    args.ws_ml[2 * (part0 + (long)hh * splits_total)] = M;
-    args.ws_ml[2 * (part0 + (long)hh * splits_total) + 1] = L;
+    if (lane < HPK) {
+      for (int ct = fc; ct <= lc; ++ct) {
+        const int sd = (cta_first_item(sp, ct) / sp.ipp) == pair ? 0 : 1;
+        const float* pp = args.partials + ((long)ct * 2 + sd) * kPart;
+        M = fmaxf(M, __ldcg(pp + lane));
+      }
+      for (int ct = fc; ct <= lc; ++ct) {
+        const int sd = (cta_first_item(sp, ct) / sp.ipp) == pair ? 0 : 1;
+        const float* pp = args.partials + ((long)ct * 2 + sd) * kPart;
+        L += __ldcg(pp + HPK + lane) * exp2f(__ldcg(pp + lane) - M);
+      }
+    }
+    for (int i = lane; i < HPK * D; i += 32) {
+      const int h = i / D;
+      const float Mh = __shfl_sync(0xffffffffu, M, h);
+      const float Lh = __shfl_sync(0xffffffffu, L, h);
+      float o = 0.f;
+      for (int ct = fc; ct <= lc; ++ct) {
+        const int sd = (cta_first_item(sp, ct) / sp.ipp) == pair ? 0 : 1;
+        const float* pp = args.partials + ((long)ct * 2 + sd) * kPart;
+        o += exp2f(__ldcg(pp + h) - Mh) * __ldcg(pp + 2 * HPK + i);
+      }
+      out[i] = o / Lh;
+    }
+    if (lane == 0) args.tickets[pair] = 0;  // ready for the next call
   }
+  (void)s_flag;
 }
 
-// out[b][h] = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s.
-// Warp 0 reads every split's (m, l) at once (two per lane, splits <= 64) and
-// reduces them with shuffles; then every thread sums its channel over the
-// splits with independent loads.
-template <int D>
-__global__ void __launch_bounds__(D) combine_kernel(DecodeArgs args, int splits) {
-  static_assert(D >= 64, "warp 0 and the split weights need D >= 64 threads");
-  __shared__ float f_s[kMaxSplitsCap];
-  __shared__ float inv_l;
-  wait_for_predecessor();  // every split's partial is written
-  allow_successor();
-  const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
-  const long part0 = ((long)b * args.Hq + h) * splits;
-  if (d < 32) {
-    float m[2], l[2];
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const int s = d + 32 * k;
-      m[k] = s < splits ? args.ws_ml[2 * (part0 + s)] : -INFINITY;
-      l[k] = s < splits ? args.ws_ml[2 * (part0 + s) + 1] : 0.f;
-    }
-    float M = fmaxf(m[0], m[1]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float L = 0.f;
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const float f = m[k] == -INFINITY ? 0.f : exp2f(m[k] - M);
-      if (d + 32 * k < splits) f_s[d + 32 * k] = f;
-      L += f * l[k];
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    if (d == 0) inv_l = 1.f / L;
-  }
-  __syncthreads();
-  const float* acc = args.ws_acc + part0 * D + d;
-  float o0 = 0.f, o1 = 0.f;
-  int s = 0;
-#pragma unroll 4
-  for (; s + 1 < splits; s += 2) {
-    o0 = fmaf(f_s[s], acc[(long)s * D], o0);
-    o1 = fmaf(f_s[s + 1], acc[(long)(s + 1) * D], o1);
-  }
-  if (s < splits) o0 = fmaf(f_s[s], acc[(long)s * D], o0);
-  args.out[((long)b * args.Hq + h) * D + d] = (o0 + o1) * inv_l;
+// ---------------------------------------------------------------------------
+// Launch
+// ---------------------------------------------------------------------------
+
+template <int D, int BITS, int HPK>
+Split make_split(int pairs, int S, int num_sms) {
+  using C = Cfg<D, BITS, HPK>;
+  Split s{};
+  s.pairs = pairs;
+  s.NG = num_groups(S);
+  const int r = S - s.NG * kGroup;
+  s.n2 = s.NG / 2;
+  s.n1 = s.NG % 2;
+  s.nr = (r + kResTok - 1) / kResTok;
+  s.ipp = s.n2 + s.n1 + s.nr;
+  s.c2 = C::kCostG2;
+  s.c1 = C::kCostG1;
+  s.cr = C::kCostR;
+  s.pc = s.n2 * s.c2 + s.n1 * s.c1 + s.nr * s.cr;
+  const long T = (long)pairs * s.pc;
+  // every CTA range must start an item: length >= the largest item cost present
+  const int cmax = max(max(s.n2 > 0 ? s.c2 : 0, s.n1 > 0 ? s.c1 : 0), s.nr > 0 ? s.cr : 0);
+  const long most = T / cmax > 0 ? T / cmax : 1;
+  int n = (int)(most < (long)min(num_sms, kGridBase) ? most : min(num_sms, kGridBase));
+  // and span at most kSlots pairs; beyond one wave, whole waves
+  const int need = (pairs + C::kSlots - 2) / (C::kSlots - 1);
+  if (need > n) n = num_sms > 0 ? (need + num_sms - 1) / num_sms * num_sms : need;
+  s.n = max(n, 1);
+  s.q = (int)(T / s.n);
+  s.rem = (int)(T % s.n);
+  return s;
 }
 
 template <int D, int BITS, int HPK>
 cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t stream) {
-  using P = Plan<D, BITS, HPK>;
-  // Per process (every device of a process is the same part): the largest
-  // shared-memory carveout, and the CTAs per SM that the kernel really gets.
-  static int ctas_per_sm = 0;
-  if (ctas_per_sm == 0) {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, BITS, HPK>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, P::kBytes);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(decode_kernel<D, BITS, HPK>,
-                             cudaFuncAttributePreferredSharedMemoryCarveout,
-                             (int)cudaSharedmemCarveoutMaxShared);
-    if (e != cudaSuccess) return e;
-    int n = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<D, BITS, HPK>, kThreads,
-                                                      P::kBytes);
-    if (e != cudaSuccess) return e;
-    ctas_per_sm = max(1, n);
-  }
-  const int NG = num_groups(a.S);
-  const int pairs = a.B * a.Hkv;
-  int splits_g = 0, gpc = 1;
-  if (NG > 0) {
-    const int want = max(1, (a.num_sms * ctas_per_sm) / pairs);   // one wave of group CTAs
-    const int by_work = max(1, NG / (2 * kWarps));                 // >= 2 groups per warp
-    splits_g = max(1, min(min(want, by_work), a.max_splits - kMaxResidualChunks));
-    gpc = (NG + splits_g - 1) / splits_g;
-    splits_g = (NG + gpc - 1) / gpc;  // every group split non-empty
-  }
-  const float qscale = (a.sm_scale > 0.f ? a.sm_scale : rsqrtf((float)D)) * kLog2e;
-  const int r = a.S - NG * kGroup;                      // residual tokens, >= 1
-  const int n_res = (r + kGroup - 1) / kGroup;           // residual chunks, <= 5
-  const int n_ctas = (splits_g + n_res) * a.Hkv * a.B;
-  cudaError_t e = launch_pdl(decode_kernel<D, BITS, HPK>, dim3(n_ctas), dim3(kThreads), P::kBytes,
-                             stream, a, splits_g, n_res, gpc, qscale);
+  using C = Cfg<D, BITS, HPK>;
+  int unused = 0;
+  cudaError_t e = per_device_setup(a.device, &unused, [](int* v) {
+    *v = 1;
+    cudaError_t r = cudaFuncSetAttribute(decode_kernel<D, BITS, HPK>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::kBytes);
+    if (r != cudaSuccess) return r;
+    return cudaFuncSetAttribute(decode_kernel<D, BITS, HPK>,
+                                cudaFuncAttributePreferredSharedMemoryCarveout,
+                                (int)cudaSharedmemCarveoutMaxShared);
+  });
   if (e != cudaSuccess) return e;
-  e = launch_pdl(combine_kernel<D>, dim3(a.Hq, a.B), dim3(D), 0, stream, a, splits_g + n_res);
+  const long pairs = (long)a.B * a.Hkv;
+  if (pairs > (1L << 30) / 4096) return cudaErrorInvalidValue;  // keeps the cost axis in int
+  const Split sp = make_split<D, BITS, HPK>((int)pairs, a.S, a.num_sms);
+  if ((long)sp.pairs * sp.pc >= (1L << 31) || sp.n > a.max_ctas) return cudaErrorInvalidValue;
+  e = launch_pdl(decode_kernel<D, BITS, HPK>, dim3(sp.n), dim3(C::kThreads), C::kBytes, stream,
+                 a, sp);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -915,10 +1226,61 @@ cudaError_t launch_decode_d(const DecodeArgs& a, cudaStream_t stream) {
   }
 }
 
+template <int D, int BITS>
+int slots_d(int hpk) {
+  switch (hpk) {
+    case 1: return Cfg<D, BITS, 1>::kSlots;
+    case 2: return Cfg<D, BITS, 2>::kSlots;
+    case 4: return Cfg<D, BITS, 4>::kSlots;
+    case 8: return Cfg<D, BITS, 8>::kSlots;
+    default: return 0;
+  }
+}
+
+template <int D, int BITS>
+int grid_d(int hpk, int pairs, int S, int num_sms) {
+  switch (hpk) {
+    case 1: return make_split<D, BITS, 1>(pairs, S, num_sms).n;
+    case 2: return make_split<D, BITS, 2>(pairs, S, num_sms).n;
+    case 4: return make_split<D, BITS, 4>(pairs, S, num_sms).n;
+    case 8: return make_split<D, BITS, 8>(pairs, S, num_sms).n;
+    default: return 0;
+  }
+}
+
+int pair_slots(int D, int bits, int hpk) {
+  if (D == 128 && bits == 2) return slots_d<128, 2>(hpk);
+  if (D == 128 && bits == 4) return slots_d<128, 4>(hpk);
+  if (D == 64 && bits == 2) return slots_d<64, 2>(hpk);
+  if (D == 64 && bits == 4) return slots_d<64, 4>(hpk);
+  return 0;
+}
+
 }  // namespace
 
+int decode_max_ctas(int D, int bits, int hpk, long pairs) {
+  const int slots = pair_slots(D, bits, hpk);
+  if (slots < 2) return 0;
+  // make_split rounds a grid above one wave up to whole waves: below 2 * need
+  const long need = (pairs + slots - 2) / (slots - 1);
+  return (int)(2 * need > kGridBase ? 2 * need : kGridBase);
+}
+
+int decode_grid_ctas(int D, int bits, int hpk, long pairs, int S, int num_sms) {
+  if (pairs < 1 || pairs > (1L << 30) / 4096 || S < 1) return 0;
+  if (D == 128 && bits == 2) return grid_d<128, 2>(hpk, (int)pairs, S, num_sms);
+  if (D == 128 && bits == 4) return grid_d<128, 4>(hpk, (int)pairs, S, num_sms);
+  if (D == 64 && bits == 2) return grid_d<64, 2>(hpk, (int)pairs, S, num_sms);
+  if (D == 64 && bits == 4) return grid_d<64, 4>(hpk, (int)pairs, S, num_sms);
+  return 0;
+}
+
+long decode_workspace_bytes(int D, int bits, int hpk, long pairs) {
+  const long ctas = decode_max_ctas(D, bits, hpk, pairs);
+  return kWsHeader + ws_tickets_bytes(pairs) + ctas * 2L * hpk * (D + 2) * (long)sizeof(float);
+}
+
 cudaError_t launch_decode(int D, int bits, const DecodeArgs& a, cudaStream_t stream) {
-  if (a.max_splits < kMaxResidualChunks + 1) return cudaErrorInvalidValue;
   if (D == 128 && bits == 2) return launch_decode_d<128, 2>(a, stream);
   if (D == 128 && bits == 4) return launch_decode_d<128, 4>(a, stream);
   if (D == 64 && bits == 2) return launch_decode_d<64, 2>(a, stream);

@@ -28,19 +28,29 @@ struct AppendArgs {
 };
 
 struct DecodeArgs {
-  const uint8_t* records;        // layer base
-  const __nv_bfloat16* ring_k;   // layer base
+  const uint8_t* records;        // layer base: [B][Hkv][ngcap] group records
+  const __nv_bfloat16* ring_k;   // layer base: [B][Hkv][R+G][D]
   const __nv_bfloat16* ring_v;
   const __nv_bfloat16* q;        // [B][Hq][D]
   float* out;                    // [B][Hq][D]
-  float* ws_ml;                  // [B][Hq][splits] x {m, l}
-  float* ws_acc;                 // [B][Hq][splits][D]
   uint32_t* status;              // device status word
+  int* tickets;                  // one per (sequence, kv head); zero between calls
+  float* partials;               // [max_ctas][2][Hq/Hkv][D + 2] split partials
+  int max_ctas;                  // capacity of `partials` in CTAs
   int B, Hkv, Hq, S, ngcap;
-  float sm_scale;
-  int max_splits;                // the workspace's capacity in splits
+  float sm_scale;                // <= 0: 1/sqrt(D)
   int num_sms;
+  int device;                    // the CUDA device the buffers live on (current at launch)
 };
+
+// Largest grid the decode kernel uses for `pairs` (sequence, kv head) pairs,
+// and the workspace bytes (status header, tickets, partials) that grid needs.
+// Host-only arithmetic; no device is queried.
+int decode_max_ctas(int D, int bits, int hpk, long pairs);
+// CTAs the decode kernel launches for this shape on a device with num_sms SMs
+// (0 for an unsupported shape).
+int decode_grid_ctas(int D, int bits, int hpk, long pairs, int S, int num_sms);
+long decode_workspace_bytes(int D, int bits, int hpk, long pairs);
 
 cudaError_t launch_prefill(int D, int bits, const PrefillArgs& a, cudaStream_t stream);
 cudaError_t launch_append(int D, int bits, const AppendArgs& a, cudaStream_t stream);

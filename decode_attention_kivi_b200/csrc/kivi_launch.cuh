@@ -9,6 +9,7 @@
 
 #include <cuda_runtime.h>
 
+#include <mutex>
 #include <utility>
 
 namespace kivi {
@@ -27,6 +28,31 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// Per-device, once-only launch set-up (function attributes such as the dynamic
+// shared-memory limit are per device).  `init(int* value)` runs once for each
+// device, with that device current, under a lock; later calls return the value
+// it produced.  Every distinct `Init` type (one lambda per kernel
+// instantiation) has its own table.
+constexpr int kMaxDevices = 64;
+
+template <typename Init>
+cudaError_t per_device_setup(int device, int* value, Init init) {
+  static std::mutex mu;
+  static bool done[kMaxDevices] = {};
+  static int values[kMaxDevices] = {};
+  if (device < 0 || device >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!done[device]) {
+    int v = 0;
+    const cudaError_t e = init(&v);
+    if (e != cudaSuccess) return e;
+    values[device] = v;
+    done[device] = true;
+  }
+  *value = values[device];
+  return cudaSuccess;
 }
 
 // Waits until the preceding kernel on the stream has completed and its writes

@@ -1,14 +1,8 @@
 // kivi_layout.cuh - geometry of the packed KIVI cache as the kernels see it.
 //
-// One group record per (layer, sequence, kv head, group of 32 tokens):
-//   K codes  [32 tokens][D*b/32 words]: channel d = code d % (32/b) of word
-//            d/(32/b); code n of a word sits at bit (n % 2)*16 + (n/2)*b (even
-//            codes in the low half, odd codes in the high half).
-//   V codes  D*32*b/32 words in the order the decode warps consume them: the
-//            word of (row group g, lane-in-quad tig, 16-channel tile mt) holds,
-//            for channels 16mt+g and 16mt+g+8, the tokens 2tig+{0,1}+{0,8}+{0,16}
-//            as (even token low half, odd token high half) pairs.  See
-//            v_code_word / v_code_bit below.
+// One group record per (layer, sequence, kv head, group of 32 tokens), in order:
+//   K codes  [32 token rows][D*b/32 words]
+//   V codes  D*32*b/32 words in the order the decode warps read them
 //   K scale  [D] fp16, K min [D] fp16
 //   V scale  [D/32][32] fp16 with the token pairs in thread order (v_meta_index),
 //   V min    the same.
@@ -16,6 +10,27 @@
 // channels ("KIVI: A Tuning-Free Asymmetric 2bit Quantization for KV Cache");
 // group size 32 and residual 128 follow the record
 // "kv-efficiency/kivi-2bit-llama3-8b-gqa-8k", field "Methodology".
+//
+// Code placement.  The decode kernel turns codes into tensor-core operands with
+// the sm_100a conversions of packed small floats: a 2-bit code c sitting in the
+// low two bits of a 4-bit field is the e2m1 value c/2, and a 4-bit code c
+// sitting in the low four bits of a byte is the e2m3 value c/8, both exact.  So
+// the 2-bit layouts put codes in the low two bits of nibbles (one mask spreads
+// eight codes into nibbles, a shifted mask the other eight), and the 4-bit
+// layouts put one code in each nibble.
+//
+//   K codes, 2 bits: channel d = 16s + 4t + j (k-step s, quad lane t, j < 4) of
+//     a token row is in word t*(D/64) + s/4 of the row, at bit
+//     8*(s%4) + 2*(j/2) + 4*(j%2).
+//   K codes, 4 bits: the same channel is in word t*(D/32) + s/2, at bit
+//     4*(s%2) + 8*j.
+//   V codes: token i, channel d of lane L = 4*(d%8) + (i%8)/2 are in lane word w
+//     (2 bits: w = d/16; 4 bits: w = 2*(d/16) + i/16), stored at word
+//     ((w/4)*32 + L)*4 + w%4, so one 16-byte load per lane and four lane words
+//     reads 512 contiguous bytes per warp.  With r = (d%16)/8, kk = i/16,
+//     hf = (i%16)/8, e = i%2 the bit is
+//       2 bits: 8*(r + 2*hf) + 2*kk + 4*e,
+//       4 bits: 8*(2*hf + e) + 4*r.
 #pragma once
 
 #include <cstdint>
@@ -26,24 +41,28 @@ constexpr int kGroup = 32;                 // G
 constexpr int kResidual = 128;             // R
 constexpr int kRingSlots = kResidual + kGroup;  // ring slots per (layer, seq, kv head)
 constexpr int kMaxHeadsPerKv = 8;
-constexpr int kMaxSplitsCap = 64;
-constexpr int kTargetCtas = 2048;          // split-K sizing target (independent of the device)
 
-// Bit offset of code n inside its 32-bit word.
-__host__ __device__ constexpr int code_bit(int n, int bits) {
-  return (n % 2) * 16 + ((n % (32 / bits)) / 2) * bits;
+// K code of channel d in a token row: word index within the row and bit offset.
+__host__ __device__ constexpr int k_code_word(int d, int D, int bits) {
+  return bits == 2 ? ((d % 16) / 4) * (D / 64) + (d / 16) / 4
+                   : ((d % 16) / 4) * (D / 32) + (d / 16) / 2;
+}
+__host__ __device__ constexpr int k_code_bit(int d, int bits) {
+  return bits == 2 ? 8 * ((d / 16) % 4) + 2 * ((d % 4) / 2) + 4 * (d % 2)
+                   : 4 * ((d / 16) % 2) + 8 * (d % 4);
 }
 
 // V code of token i (0..31), channel d: word index and bit offset.
-__host__ __device__ constexpr int v_code_idx(int i, int d) {
-  return 4 * (i / 16) + 2 * ((i % 16) / 8) + (d % 16) / 8;  // 4 kk + 2 hf + r
+__host__ __device__ constexpr int v_lane_word(int i, int d, int bits) {
+  return bits == 2 ? d / 16 : 2 * (d / 16) + i / 16;
 }
-__host__ __device__ constexpr int v_code_word(int i, int d, int D, int bits) {
-  return ((4 * (d % 8) + (i % 8) / 2) * (D / 16) + d / 16) * (bits / 2) +
-         v_code_idx(i, d) / (16 / bits);
+__host__ __device__ constexpr int v_code_word(int i, int d, int bits) {
+  return ((v_lane_word(i, d, bits) / 4) * 32 + 4 * (d % 8) + (i % 8) / 2) * 4 +
+         v_lane_word(i, d, bits) % 4;
 }
 __host__ __device__ constexpr int v_code_bit(int i, int d, int bits) {
-  return 16 * (i % 2) + (v_code_idx(i, d) % (16 / bits)) * bits;
+  return bits == 2 ? 8 * ((d % 16) / 8 + 2 * ((i % 16) / 8)) + 2 * (i / 16) + 4 * (i % 2)
+                   : 8 * (2 * ((i % 16) / 8) + i % 2) + 4 * ((d % 16) / 8);
 }
 // fp16 index of the V scale / min of token i, channel block j.
 __host__ __device__ constexpr int v_meta_index(int i, int j) {
@@ -56,9 +75,7 @@ __host__ __device__ constexpr int num_groups(int S) {
 
 struct RecordGeom {
   int D, bits;
-  __host__ __device__ constexpr int codes_per_word() const { return 32 / bits; }
   __host__ __device__ constexpr int k_row_words() const { return D * bits / 32; }
-  __host__ __device__ constexpr int v_row_words() const { return kGroup * bits / 32; }
   __host__ __device__ constexpr int code_words() const { return kGroup * D * bits / 32; }
   __host__ __device__ constexpr long k_codes_off() const { return 0; }
   __host__ __device__ constexpr long v_codes_off() const { return 4L * code_words(); }
@@ -69,18 +86,12 @@ struct RecordGeom {
   __host__ __device__ constexpr long bytes() const { return v_min_off() + 2L * D; }
 };
 
-// Split-K partials per (sequence, query head) the workspace is sized for: at
-// least one split over the quantized groups plus one per residual chunk of up
-// to 32 tokens (the residual holds fewer than R + G = 160 tokens: 5 chunks).
-constexpr int kMinSplits = 1 + (kRingSlots + kGroup - 1) / kGroup;
-__host__ __device__ constexpr int max_splits(int batch, int kv_heads) {
-  int pairs = batch * kv_heads;
-  int s = (kTargetCtas + pairs - 1) / pairs;
-  return s < kMinSplits ? kMinSplits : (s > kMaxSplitsCap ? kMaxSplitsCap : s);
-}
-
-// Workspace: [0, 256) device status word and padding; then per (b, q head,
-// split) the running max m and sum l (two floats), then acc[D] floats.
+// Workspace of a handle (and of the static scratch array): [0, 256) the device
+// status word and padding; then one int ticket per (sequence, kv head), rounded
+// up to 256 bytes; then the split partials of the decode kernel.
 constexpr long kWsHeader = 256;
+__host__ __device__ constexpr long ws_tickets_bytes(long pairs) {
+  return (4 * pairs + 255) / 256 * 256;
+}
 
 }  // namespace kivi

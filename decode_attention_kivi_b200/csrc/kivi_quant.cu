@@ -59,7 +59,6 @@ template <int D, int BITS>
 __device__ void quantize_tiles_to_record(QuantSmem<D>& sm, uint32_t* __restrict__ rec) {
   constexpr RecordGeom geo{D, BITS};
   constexpr int kQmax = (1 << BITS) - 1;
-  constexpr int kCpw = geo.codes_per_word();
   unsigned short* rec16 = reinterpret_cast<unsigned short*>(rec);
   unsigned short* kscale = rec16 + geo.k_scale_off() / 2;
   unsigned short* kmin = rec16 + geo.k_min_off() / 2;
@@ -99,33 +98,44 @@ __device__ void quantize_tiles_to_record(QuantSmem<D>& sm, uint32_t* __restrict_
     vmin[v_meta_index(t, j)] = to_f16_bits(mn);
   }
   __syncthreads();
-  // Pack: K token-major rows (channels innermost), V channel-major rows (tokens innermost).
-  constexpr int kWords = geo.code_words();
-  for (int wi = threadIdx.x; wi < kWords; wi += kQuantThreads) {
+  // Pack the K codes: word w of token row t.  The word belongs to quad lane
+  // tq = w / (D*b/128) and covers k-steps s = (32/(4b)) * (w % (D*b/128)) + sl;
+  // code j of k-step s is channel 16s + 4tq + j (see kivi_layout.cuh).
+  constexpr int kLaneWords = D * BITS / 128;  // words of one quad lane in a row
+  constexpr int kStepsPerWord = 8 / BITS;
+  for (int wi = threadIdx.x; wi < geo.code_words(); wi += kQuantThreads) {
     const int t = wi / geo.k_row_words(), w = wi % geo.k_row_words();
+    const int tq = w / kLaneWords, s0 = kStepsPerWord * (w % kLaneWords);
     uint32_t word = 0;
 #pragma unroll
-    for (int i = 0; i < kCpw; ++i) word |= (uint32_t)sm.kc[t][w * kCpw + i] << code_bit(i, BITS);
+    for (int sl = 0; sl < kStepsPerWord; ++sl)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int d = 16 * (s0 + sl) + 4 * tq + j;
+        word |= (uint32_t)sm.kc[t][d] << k_code_bit(d, BITS);
+      }
     rec[wi] = word;
   }
-  // V: word wi belongs to (g, tig, mt) = its block of BITS/2 words; each word
-  // holds 16/BITS pairs idx = 4kk + 2hf + r of tokens 16kk+8hf+2tig+{0,1} of
-  // channel 16mt+g+8r (inverse of v_code_word / v_code_bit).
-  constexpr int kWordsPer = BITS / 2, kPairs = 16 / BITS;
-  for (int wi = threadIdx.x; wi < kWords; wi += kQuantThreads) {
-    const int base = wi / kWordsPer, w2 = wi % kWordsPer;
-    const int mt = base % (D / 16), gt = base / (D / 16);
-    const int g = gt / 4, tig = gt % 4;
+  // Pack the V codes: stored word wi holds lane word w of lane L = 4g + tig
+  // (inverse of v_code_word); its codes are channels 16mt + g + 8r of tokens
+  // 16kk + 8hf + 2tig + e.
+  for (int wi = threadIdx.x; wi < geo.code_words(); wi += kQuantThreads) {
+    const int L = (wi % 128) / 4, w = (wi / 128) * 4 + wi % 4;
+    const int g = L / 4, tig = L % 4;
     uint32_t word = 0;
 #pragma unroll
-    for (int p = 0; p < kPairs; ++p) {
-      const int idx = w2 * kPairs + p;
-      const int kk = idx / 4, hf = (idx / 2) % 2, r = idx % 2;
-      const int d = 16 * mt + g + 8 * r;
-      const int t0 = 16 * kk + 8 * hf + 2 * tig;
-      word |= (uint32_t)sm.vc[t0][d] << (p * BITS);
-      word |= (uint32_t)sm.vc[t0 + 1][d] << (16 + p * BITS);
-    }
+    for (int kk = 0; kk < 2; ++kk)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int mt = BITS == 2 ? w : w / 2;
+            if (BITS == 4 && kk != w % 2) continue;
+            const int d = 16 * mt + g + 8 * r, i = 16 * kk + 8 * hf + 2 * tig + e;
+            word |= (uint32_t)sm.vc[i][d] << v_code_bit(i, d, BITS);
+          }
     rec[geo.v_codes_off() / 4 + wi] = word;
   }
 }

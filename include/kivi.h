@@ -209,6 +209,16 @@ kivi_status kivi_decode_attention_static_scratch(const kivi_config* cfg, const v
                                                  int32_t layer, int32_t S, const void* q,
                                                  float* out, float sm_scale, void* stream);
 
+/* The device status word of kivi_decode_attention_static_scratch on the current
+ * device (that call keeps it in the static scratch array, not in a workspace):
+ * synchronises `stream`, reads the word through the array's device address
+ * and clears it.  Returns KIVI_ERR_DEVICE if one of those calls recorded a
+ * failure (a bounded wait that ran out) since the last query, KIVI_ERR_CUDA if
+ * a CUDA call failed, else KIVI_OK.  `code_out` (may be NULL) receives the raw
+ * word.  Allocates nothing; like the attention call, its first use on a device
+ * looks up the array's address.  The pages have no counterpart. */
+kivi_status kivi_static_scratch_status(void* stream, uint32_t* code_out);
+
 /* Synchronises `stream`, then reads and clears the device status word.
  * Returns KIVI_ERR_DEVICE if a kernel recorded a failure (a bounded wait that
  * ran out), KIVI_ERR_CUDA if the synchronisation failed, else KIVI_OK.

@@ -136,34 +136,55 @@ int oracle_num_groups(int S) {
   return (S - ORACLE_R) / ORACLE_G;
 }
 
-/* Code `index` of a row goes to word index / (32/b); inside the word the
- * even-indexed codes fill the low 16 bits and the odd-indexed codes the high 16
- * bits, each half from its least significant bit: bit offset
- * (index mod 2) * 16 + ((index mod (32/b)) / 2) * b. */
-static int code_bit_offset(int index, int bits) {
-  int in_word = index % (32 / bits);
-  return (in_word % 2) * 16 + (in_word / 2) * bits;
+/* Key codes of one token row: D*b/32 little-endian 32-bit words.  The decode
+ * kernel walks the channels in k-steps of 16 and hands channel
+ * d = 16 s + 4 t + j (k-step s, quad lane t = 0..3, j = 0..3) to quad lane t,
+ * which owns the W = D*b/128 words t*W .. t*W + W - 1 of the row; each of those
+ * words covers 8/b consecutive k-steps, the k-step s being number
+ * s mod (8/b) inside its word.
+ *   2 bits: byte (s mod 4) of the word holds the four codes of k-step s: j = 0
+ *           in bits 0-1, j = 1 in bits 4-5, j = 2 in bits 2-3, j = 3 in bits
+ *           6-7 (each code in the low half of a nibble).
+ *   4 bits: byte j of the word holds code j of the word's first k-step in its
+ *           low nibble and of its second k-step in its high nibble. */
+static void k_code_position(int d, int D, int bits, int* word_in_row, int* bit) {
+  const int s = d / 16, t = (d % 16) / 4, j = d % 4;
+  const int per_word = 8 / bits; /* k-steps per word */
+  *word_in_row = t * (D * bits / 128) + s / per_word;
+  if (bits == 2) {
+    static const int nibble_offset[4] = {0, 4, 2, 6};
+    *bit = 8 * (s % per_word) + nibble_offset[j];
+  } else {
+    *bit = 8 * j + 4 * (s % per_word);
+  }
 }
 
-static void put_code(uint32_t* words, int index, int bits, int code) {
-  words[index / (32 / bits)] |= (uint32_t)code << code_bit_offset(index, bits);
+static void put_key_code(uint32_t* row_words, int d, int D, int bits, int code) {
+  int w, b;
+  k_code_position(d, D, bits, &w, &b);
+  row_words[w] |= (uint32_t)code << b;
 }
 
-/* Value codes are stored in the order the decode kernel's threads consume
- * them.  For token i (0..31) and channel d of a group record:
- *   mt = d / 16, g = d mod 8, r = (d mod 16) / 8,
- *   kk = i / 16, hf = (i mod 16) / 8, tig = (i mod 8) / 2, e = i mod 2,
- *   idx = 4 kk + 2 hf + r, p = 16 / b pairs per word,
- *   word = ((4 g + tig) * (D / 16) + mt) * (b / 2) + idx / p,
- *   bit  = 16 e + (idx mod p) * b.
- * So each word holds, for channels d and d + 8, pairs of adjacent tokens with
- * the even token in the low 16 bits and the odd token in the high 16 bits. */
+/* Value codes are stored in the order the decode kernel's threads read them.
+ * Token i (0..31), channel d of a group record belong to lane
+ * L = 4 (d mod 8) + (i mod 8) / 2 and to that lane's word
+ *   lw = d / 16            (2 bits),
+ *   lw = 2 (d / 16) + i/16 (4 bits);
+ * lane words are interleaved four at a time over the 32 lanes:
+ *   word = ((lw / 4) * 32 + L) * 4 + lw mod 4.
+ * Inside the word, with r = (d mod 16) / 8, kk = i / 16, hf = (i mod 16) / 8,
+ * e = i mod 2:
+ *   2 bits: bit 8 (r + 2 hf) + 2 kk + 4 e (nibble pairs: even token low, odd
+ *           token high),
+ *   4 bits: bit 8 (2 hf + e) + 4 r (one code per nibble). */
 static void v_code_position(int i, int d, int D, int bits, long* word, int* bit) {
+  (void)D;
   const int mt = d / 16, g = d % 8, r = (d % 16) / 8;
   const int kk = i / 16, hf = (i % 16) / 8, tig = (i % 8) / 2, e = i % 2;
-  const int idx = 4 * kk + 2 * hf + r, per_word = 16 / bits;
-  *word = ((long)(4 * g + tig) * (D / 16) + mt) * (bits / 2) + idx / per_word;
-  *bit = 16 * e + (idx % per_word) * bits;
+  const int lane = 4 * g + tig;
+  const int lw = bits == 2 ? mt : 2 * mt + kk;
+  *word = ((long)(lw / 4) * 32 + lane) * 4 + lw % 4;
+  *bit = bits == 2 ? 8 * (r + 2 * hf) + 2 * kk + 4 * e : 8 * (2 * hf + e) + 4 * r;
 }
 
 /* fp16 index of the value scale (and min) of token i, channel block j: each
@@ -209,7 +230,7 @@ void oracle_make_record(const uint16_t* k, const uint16_t* v, long ld, int D,
     float scale, mn;
     oracle_quantize_group(col, G, 1, bits, &scale, &mn, codes);
     /* token-major rows of D*b/32 words: channel d of token i */
-    for (int i = 0; i < G; ++i) put_code(kcodes + (long)i * D * bits / 32, d, bits, codes[i]);
+    for (int i = 0; i < G; ++i) put_key_code(kcodes + (long)i * D * bits / 32, d, D, bits, codes[i]);
     put_u16(kscale + 2L * d, oracle_f32_to_f16_bits(scale));
     put_u16(kmin + 2L * d, oracle_f32_to_f16_bits(mn));
   }
@@ -241,13 +262,14 @@ void oracle_make_record(const uint16_t* k, const uint16_t* v, long ld, int D,
   free(vcodes);
 }
 
-/* Reads code `index` of a packed little-endian word row. */
-static int get_code(const uint8_t* row, int index, int bits) {
-  int per_word = 32 / bits;
-  const uint8_t* w = row + 4L * (index / per_word);
-  uint32_t word = (uint32_t)w[0] | ((uint32_t)w[1] << 8) | ((uint32_t)w[2] << 16) |
-                  ((uint32_t)w[3] << 24);
-  return (int)((word >> code_bit_offset(index, bits)) & ((1u << bits) - 1u));
+/* Reads the key code of channel d from a packed little-endian token row. */
+static int get_key_code(const uint8_t* row, int d, int D, int bits) {
+  int w, b;
+  k_code_position(d, D, bits, &w, &b);
+  const uint8_t* p = row + 4L * w;
+  uint32_t word = (uint32_t)p[0] | ((uint32_t)p[1] << 8) | ((uint32_t)p[2] << 16) |
+                  ((uint32_t)p[3] << 24);
+  return (int)((word >> b) & ((1u << bits) - 1u));
 }
 
 static uint16_t get_u16(const uint8_t* p) { return (uint16_t)(p[0] | (p[1] << 8)); }
@@ -265,7 +287,7 @@ void oracle_dequant_record(const uint8_t* record, int D, int bits, double* k_hat
   const uint8_t* vmin = vscale + 2L * D;
   for (int i = 0; i < G; ++i) {
     for (int d = 0; d < D; ++d) {
-      int ck = get_code(record + 4L * row_words_k * i, d, bits);
+      int ck = get_key_code(record + 4L * row_words_k * i, d, D, bits);
       double sk = oracle_f16_bits_to_double(get_u16(kscale + 2L * d));
       double mk = oracle_f16_bits_to_double(get_u16(kmin + 2L * d));
       k_hat[(long)i * D + d] = sk * ck + mk;

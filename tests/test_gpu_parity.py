@@ -15,48 +15,16 @@ import torch
 
 import oracle as O
 import synth
+from gpu_util import assert_attention_close, assert_state_equal, load_kivi
 
 pytestmark = pytest.mark.gpu
-
-ATOL = 2e-3
-RTOL = 2e-3
 
 
 @pytest.fixture(scope="module")
 def kivi():
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
-    from decode_attention_kivi_b200 import build
-
-    build.build()
-    import decode_attention_kivi_b200 as K
-
-    return K
-
-
-def assert_attention_close(gpu: np.ndarray, ref: np.ndarray, what=""):
-    err = np.abs(gpu.astype(np.float64) - ref)
-    bound = ATOL + RTOL * np.abs(ref)
-    bad = err > bound
-    assert not np.isnan(gpu).any(), f"{what}: NaN in GPU output"
-    assert not bad.any(), (f"{what}: {bad.sum()} of {bad.size} outside tolerance, "
-                           f"max err {err.max():.3e} at {np.unravel_index(err.argmax(), err.shape)}")
-
-
-def assert_state_equal(cache, layer, ref: O.OracleCache, what=""):
-    S, NG = cache.length(layer)
-    assert (S, NG) == (ref.S, ref.NG), what
-    if NG:
-        got = cache.records_view(layer)[:, :, :NG].cpu().numpy()
-        exp = ref.records[:, :, :NG]
-        if not np.array_equal(got, exp):
-            diff = np.argwhere(got != exp)
-            raise AssertionError(f"{what}: {len(diff)} record bytes differ, first at {diff[0]}")
-    for t in range(NG * O.G, S):
-        slot = t % (O.R + O.G)
-        for which, arr in (("k", ref.ring_k), ("v", ref.ring_v)):
-            got = synth.bf16_bits(cache.ring_view(which, layer)[:, :, slot])
-            assert np.array_equal(got, arr[:, :, slot]), f"{what}: ring {which} token {t}"
+    return load_kivi()
 
 
 def _rand(shape, gen, scale=None):

@@ -163,7 +163,7 @@ def test_packed_words_hand_worked(bits):
         assert _word(rec, row_bytes_k) == int(g["2bit_k_row1_word0"], 16)
     else:
         assert _word(rec, 0) == int(g["4bit_k_row0_word0"], 16)
-        assert _word(rec, 4) == int(g["4bit_k_row0_word1"], 16)
+        assert _word(rec, 16) == int(g["4bit_k_row0_word4"], 16)
         assert _word(rec, row_bytes_k) == int(g["4bit_k_row1_word0"], 16)
     kscale = 2 * 32 * row_bytes_k
     kmin, vscale = kscale + 2 * D, kscale + 4 * D

@@ -4,7 +4,9 @@ from __future__ import annotations
 import ctypes
 import os
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkivi.so")
+# KIVI_LIBRARY selects another in-tree build (the debug library in its tests)
+_LIB_PATH = os.environ.get("KIVI_LIBRARY") or os.path.join(
+    os.path.dirname(os.path.abspath(__file__)), "libkivi.so")
 
 
 class KiviConfig(ctypes.Structure):
@@ -65,6 +67,8 @@ def lib() -> ctypes.CDLL:
                                                       I32, P, P, F32, P]),
         "kivi_static_scratch_status": (st, [P, ctypes.POINTER(ctypes.c_uint32)]),
     }
+    if hasattr(L, "kivi_debug_overstate_copies"):  # debug build only
+        sig["kivi_debug_overstate_copies"] = (st, [ctypes.c_uint32])
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
         fn.restype = res

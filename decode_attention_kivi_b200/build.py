@@ -9,6 +9,9 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libkivi.so")
+DEBUG_LIB = os.path.join(PKG, "libkivi_debug.so")
+# debug build: short bounded waits (about 1 ms), copy bounds checks, a test hook
+DEBUG_FLAGS = ["-DKIVI_DEBUG_BUILD", "-DKIVI_DEBUG_BOUNDS", "-DKIVI_DEBUG_WAIT_CYCLES=2000000LL"]
 SOURCES = ["kivi_api.cu", "kivi_quant.cu", "kivi_attn.cu"]
 NVCC_FLAGS = [
     "-O3", "-std=c++17",
@@ -25,26 +28,28 @@ def _inputs():
     return files + [os.path.join(ROOT, "include", "kivi.h")]
 
 
-def stale() -> bool:
-    if not os.path.exists(LIB):
+def stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(f) > t for f in _inputs())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not stale():
-        return LIB
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    """Builds libkivi.so (or, with debug=True, libkivi_debug.so) when stale."""
+    lib = DEBUG_LIB if debug else LIB
+    if not force and not stale(lib):
+        return lib
     nvcc = os.environ.get("NVCC", "nvcc")
-    tmp = LIB + ".tmp"
-    cmd = [nvcc, *NVCC_FLAGS, "-o", tmp, *[os.path.join(CSRC, s) for s in SOURCES]]
+    tmp = lib + ".tmp"
+    cmd = [nvcc, *NVCC_FLAGS, *(DEBUG_FLAGS if debug else []), "-o", tmp,
+           *[os.path.join(CSRC, s) for s in SOURCES]]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose=True, debug="--debug" in sys.argv))

@@ -63,17 +63,25 @@ kivi_sizes sizes_of(const kivi_config* c) {
 }
 
 long partial_bytes(const kivi_config* c) {
-  return 2L * (c->num_q_heads / c->num_kv_heads) * (c->head_dim + 2) * (long)sizeof(float);
+  return kivi::decode_partial_bytes(c->head_dim, c->num_q_heads / c->num_kv_heads);
+}
+
+// Bytes before the partials: status header, tickets, parked warp states.
+long fixed_workspace_bytes(const kivi_config* c) {
+  const long pairs = (long)c->batch * c->num_kv_heads;
+  return kivi::kWsHeader + kivi::ws_tickets_bytes(pairs) +
+         kivi::decode_parks_bytes(c->head_dim, c->num_q_heads / c->num_kv_heads, pairs);
 }
 
 // Points the decode arguments at a workspace of `bytes` bytes: status header,
-// tickets, then as many CTAs' partials as fit.
+// tickets, parked warp states, then as many CTAs' partials as fit.
 void bind_workspace(kivi::DecodeArgs& a, const kivi_config* c, void* ws, size_t bytes) {
   const long pairs = (long)c->batch * c->num_kv_heads;
   uint8_t* base = static_cast<uint8_t*>(ws);
-  const long fixed = kivi::kWsHeader + kivi::ws_tickets_bytes(pairs);
+  const long fixed = fixed_workspace_bytes(c);
   a.status = reinterpret_cast<uint32_t*>(base);
   a.tickets = reinterpret_cast<int*>(base + kivi::kWsHeader);
+  a.parks = reinterpret_cast<float*>(base + kivi::kWsHeader + kivi::ws_tickets_bytes(pairs));
   a.partials = reinterpret_cast<float*>(base + fixed);
   const long room = (long)bytes - fixed;
   a.max_ctas = room > 0 ? (int)(room / partial_bytes(c)) : 0;
@@ -375,8 +383,8 @@ extern "C" kivi_status kivi_decode_attention_static_scratch(
   const long pairs = (long)cfg->batch * cfg->num_kv_heads;
   const int hpk = cfg->num_q_heads / cfg->num_kv_heads;
 
-  // the fixed part (status word, tickets) must fit before any device work
-  const long fixed = kivi::kWsHeader + kivi::ws_tickets_bytes(pairs);
+  // the fixed part (status word, tickets, parked states) must fit before any device work
+  const long fixed = fixed_workspace_bytes(cfg);
   if (fixed + partial_bytes(cfg) > (long)KIVI_STATIC_SCRATCH_BYTES) return KIVI_ERR_SCRATCH_LIMIT;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -425,3 +433,11 @@ extern "C" kivi_status kivi_static_scratch_status(void* stream, uint32_t* code_o
   if (code_out) *code_out = code;
   return code ? KIVI_ERR_DEVICE : KIVI_OK;
 }
+
+#ifdef KIVI_DEBUG_BUILD
+#include "../../include/kivi_debug.h"
+
+extern "C" kivi_status kivi_debug_overstate_copies(uint32_t bytes) {
+  return from_cuda(kivi::debug_overstate_copies(bytes));
+}
+#endif

@@ -58,15 +58,33 @@ namespace kivi {
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
+#ifdef KIVI_DEBUG_WAIT_CYCLES
+constexpr long long kWaitBudgetCycles = KIVI_DEBUG_WAIT_CYCLES;  // debug build: short waits
+#else
 constexpr long long kWaitBudgetCycles = 4000000000LL;  // about 2 s at 1.9 GHz
-constexpr int kLockSpinLimit = 1 << 24;
+#endif
 constexpr uint32_t kStatusWaitTimeout = 1u;
-constexpr uint32_t kStatusLockTimeout = 2u;
 constexpr uint32_t kStatusBadSplit = 4u;
+constexpr uint32_t kStatusBounds = 8u;  // debug build: an index outside its buffer (access skipped)
+
+#ifdef KIVI_DEBUG_BUILD
+// Debug build only: bytes added to every expected copy size, so that a test can
+// make the bounded waits run out while every issued copy still lands whole.
+__device__ unsigned g_kivi_debug_overstate = 0u;
+__device__ __forceinline__ uint32_t debug_overstate() { return g_kivi_debug_overstate; }
+#else
+__device__ __forceinline__ uint32_t debug_overstate() { return 0u; }
+#endif
 constexpr int kResTok = 8;             // residual tokens per item
 constexpr int kPRow = 2 * 32 + 8;      // p tile row (fp16 entries): 64 tokens + 8 padding
 constexpr int kGridBase = 256;         // CTAs at most, before the pair-slot bound
 constexpr int kSmemBudget = 227 * 1024;
+#ifndef KIVI_ITEM_SLOTS
+#define KIVI_ITEM_SLOTS 2
+#endif
+#ifndef KIVI_MAX_WARPS
+#define KIVI_MAX_WARPS 16
+#endif
 
 // ---------------------------------------------------------------------------
 // PTX wrappers
@@ -295,6 +313,7 @@ struct Cfg {
   static constexpr RecordGeom geo{D, BITS};
   static constexpr int kRec = (int)geo.bytes();          // multiple of 128
   static constexpr int kItemBytes = 2 * kRec;             // two records, or 8 K + 8 V rows
+  static constexpr int kItemSlots = KIVI_ITEM_SLOTS;        // items in a warp's ring
   static constexpr int kResRow = 2 * D + 16;              // padded residual row (bank spread)
   static_assert(kResTok * kResRow <= kRec, "residual rows must fit in one record's space");
   static constexpr int kChunks = HPK > 4 ? 2 : 1;         // score column chunks of 4 heads
@@ -303,17 +322,20 @@ struct Cfg {
   // p tile rows: heads' p_hi, then -p_lo (<= 4 heads) or p_lo (8 heads), then a zero row
   static constexpr int kPRows = 2 * HPK + (kLoCols ? 1 : 0);
   static constexpr int kZeroRow = 2 * HPK;
-  static constexpr int kWarpBytes = round_up(2 * kItemBytes + kPRows * kPRow * 2, 128);
-  static constexpr int kSlotBytes = round_up(96 + HPK * D * 4 + HPK * D * 2, 16);  // merge + q
+  static constexpr int kWarpBytes = round_up(kItemSlots * kItemBytes + kPRows * kPRow * 2, 128);
+  static constexpr int kSlotBytes = HPK * D * 2;          // a pair's q (bf16)
+  static constexpr int kStateFloats = HPK * (D + 2);      // m[HPK], l[HPK], acc[HPK][D]
+  static_assert(kStateFloats * 4 <= kItemSlots * kItemBytes, "a warp's final state fits its item slots");
   static constexpr int kMinSlots = 4;
-  static constexpr int kFixed = 512;                      // mbarriers (16 B a warp), counter
+  static constexpr int kFixed = 2048;                     // mbarriers, counters, masks
   static constexpr int kNW =
-      HPK > 4 ? 8 : cmin_i(16, (kSmemBudget - kFixed - kMinSlots * kSlotBytes) / kWarpBytes);
+      cmin_i(HPK > 4 ? cmin_i(8, KIVI_MAX_WARPS) : KIVI_MAX_WARPS,
+             (kSmemBudget - kFixed - kMinSlots * kSlotBytes) / kWarpBytes);
   static constexpr int kThreads = kNW * 32;
   static constexpr int kSlots =
       cmin_i(64, (kSmemBudget - kFixed - kNW * kWarpBytes) / kSlotBytes);
   static_assert(kNW >= 4 && kSlots >= kMinSlots, "shared-memory plan");
-  static_assert(16 * kNW + 8 <= kFixed, "mbarriers and the claim counter fit the fixed area");
+  static_assert(8 * kItemSlots * kNW + 16 + 8 * kNW + 12 * kSlots <= kFixed, "fixed area");
   static constexpr int kOffSlots = kNW * kWarpBytes;
   static constexpr int kOffFixed = kOffSlots + kSlots * kSlotBytes;
   static constexpr int kBytes = kOffFixed + kFixed;
@@ -323,16 +345,12 @@ struct Cfg {
   static constexpr int kCostR = kResTok * D * 4 / 512 + 1;
 };
 
-// One pair slot of a CTA: merged online-softmax state and the pair's q.
-template <int D, int HPK>
-struct PairSlot {
-  float m[8];
-  float l[8];
-  int lock;
-  int pad[7];
-  float acc[HPK][D];
-  __nv_bfloat16 q[HPK][D];
-};
+// Parked warp states: one slot per (pair, warp) of up to kParkWarps warps, each
+// state m[HPK], l[HPK], acc[HPK][D] in fp32, padded to whole 128-byte lines.
+constexpr int kParkWarps = 16;
+__host__ __device__ constexpr long park_stride_floats(int D, int hpk) {
+  return ((long)hpk * (D + 2) * 4 + 127) / 128 * 32;
+}
 
 // ---------------------------------------------------------------------------
 // The split of the items between CTAs
@@ -346,7 +364,14 @@ struct Split {
   int pairs, ipp, n2, n1, nr, NG;
   int c2, c1, cr, pc;  // item costs, cost per pair
   int n, q, rem;       // CTAs and the division of pairs*pc among them
+  unsigned long long ipp_inv;  // ceil(2^64 / ipp) for ipp >= 2: x / ipp = umulhi64(x, ipp_inv)
 };
+
+// Pair of global item `it` (0 <= it < 2^31): one 64-bit high multiply instead of
+// a division by the runtime value ipp.
+__device__ __forceinline__ int pair_of(const Split& s, int it) {
+  return s.ipp == 1 ? it : (int)__umul64hi((unsigned long long)it, s.ipp_inv);
+}
 
 __host__ __device__ inline int cost_lo(const Split& s, int c) {
   return c * s.q + (c < s.rem ? c : s.rem);
@@ -372,13 +397,19 @@ __host__ __device__ inline int cta_first_item(const Split& s, int c) {
   return first_item_at(s, cost_lo(s, c));
 }
 
-// The CTA that owns global item `it`.
-__host__ __device__ inline int cta_of_item(const Split& s, int it) {
+// Start of global item `it` (it <= pairs * ipp) on the cost axis.
+__host__ __device__ inline int item_cost_start(const Split& s, int it) {
   const int p = it / s.ipp, k = it % s.ipp;
   int cs = p * s.pc;
   if (k <= s.n2) cs += k * s.c2;
   else if (k <= s.n2 + s.n1) cs += s.n2 * s.c2 + (k - s.n2) * s.c1;
   else cs += s.n2 * s.c2 + s.n1 * s.c1 + (k - s.n2 - s.n1) * s.cr;
+  return cs;
+}
+
+// The CTA that owns global item `it`.
+__host__ __device__ inline int cta_of_item(const Split& s, int it) {
+  const int cs = item_cost_start(s, it);
   const int big = s.rem * (s.q + 1);
   return cs < big ? cs / (s.q + 1) : s.rem + (cs - big) / s.q;
 }
@@ -412,7 +443,7 @@ struct Warp {
   uint32_t qa[kChunks][kKSteps][2], qb[kChunks][kKSteps][2];
   float ch[kChunks];      // log2 score scale of head 4c + tig
   float qscale;           // sm_scale * log2(e)
-  const __nv_bfloat16* q_pair;  // the pair's q (HPK x D) in shared memory
+  const __nv_bfloat16* q_pair;  // the pair's q (HPK x D, global memory)
   unsigned char* p_tile;  // this warp's p tile
   int rowA, rowX, rowR;   // p tile rows this lane reads (byte offsets)
   uint32_t maskY, signY, maskHi;
@@ -818,8 +849,6 @@ __global__ void __launch_bounds__(Cfg<D, BITS, HPK>::kThreads, 1)
 decode_kernel(DecodeArgs args, Split sp) {
   using C = Cfg<D, BITS, HPK>;
   using W = Warp<D, BITS, HPK>;
-  using Slot = PairSlot<D, HPK>;
-  static_assert(sizeof(Slot) <= C::kSlotBytes, "pair slot size");
   extern __shared__ __align__(128) unsigned char smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cta = blockIdx.x;
@@ -828,49 +857,129 @@ decode_kernel(DecodeArgs args, Split sp) {
   const int p_first = it_begin / sp.ipp, p_last = (it_end - 1) / sp.ipp;
   const int n_pairs = p_last - p_first + 1;
   unsigned char* wbase = smem + warp * C::kWarpBytes;
-  Slot* slots = reinterpret_cast<Slot*>(smem + C::kOffSlots);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffFixed) + 2 * warp;
-  int* s_ctr = reinterpret_cast<int*>(smem + C::kOffFixed + 8 * 2 * C::kNW);
-  int* s_flag = s_ctr + 1;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffFixed) + C::kItemSlots * warp;
+  int* s_ctr = reinterpret_cast<int*>(smem + C::kOffFixed + 8 * C::kItemSlots * C::kNW);
+  int* s_final = s_ctr + 4;                          // [kNW] pair (local) of each warp's final state
+  unsigned* s_parked = reinterpret_cast<unsigned*>(s_final + C::kNW);  // [kSlots] warp bitmasks
+  int* s_seg_next = reinterpret_cast<int*>(s_parked + C::kSlots);      // [kSlots] claim counters
+  int* s_seg_end = s_seg_next + C::kSlots;                             // [kSlots] end items
   if (it_end <= it_begin || n_pairs > C::kSlots) {  // the host's split rules exclude both
     if (threadIdx.x == 0) atomicOr(args.status, kStatusBadSplit);
     return;
   }
 
-  // ---- set-up: p tiles, mbarriers, pair slots, the claim counter ----
+  // ---- set-up: p tiles, mbarriers, masks, the claim counter ----
   {
-    uint32_t* pt = reinterpret_cast<uint32_t*>(wbase + 2 * C::kItemBytes);
+    uint32_t* pt = reinterpret_cast<uint32_t*>(wbase + C::kItemSlots * C::kItemBytes);
     for (int i = lane; i < C::kPRows * kPRow / 2; i += 32) pt[i] = 0u;
     if (lane == 0) {
-      mbar_init(&bars[0], 1);
-      mbar_init(&bars[1], 1);
+      for (int k = 0; k < C::kItemSlots; ++k) mbar_init(&bars[k], 1);
       fence_mbar_init();
+      s_final[warp] = -1;
     }
-    for (int k = warp; k < n_pairs; k += C::kNW) {
-      Slot& sl = slots[k];
-      if (lane < 8) {
-        sl.m[lane] = -INFINITY;
-        sl.l[lane] = 0.f;
+    for (int k = threadIdx.x; k < n_pairs; k += C::kThreads) {
+      s_parked[k] = 0u;
+      s_seg_next[k] = max(it_begin, (p_first + k) * sp.ipp);
+      s_seg_end[k] = min(it_end, (p_first + k + 1) * sp.ipp);
+    }
+  }
+  // Segments: the items of one pair inside this CTA's range.  With at most kNW
+  // segments every segment gets its own group of warps, sized by its cost, so a
+  // warp never leaves its pair; with more, each warp sweeps a run of segments.
+  // Thread 0 writes each warp's segment range [lo, hi) to s_warp_seg.
+  int* s_warp_seg = s_seg_end + C::kSlots;  // [kNW]: lo | hi << 16
+  if (threadIdx.x == 0) {
+    if (n_pairs <= C::kNW) {
+      int cost[C::kNW], wk[C::kNW];
+      for (int k = 0; k < n_pairs; ++k) {
+        const int a = max(it_begin, (p_first + k) * sp.ipp);
+        const int b = min(it_end, (p_first + k + 1) * sp.ipp);
+        cost[k] = item_cost_start(sp, b) - item_cost_start(sp, a);
+        wk[k] = 1;
       }
-      if (lane == 0) sl.lock = 0;
-      for (int i = lane; i < HPK * D; i += 32) (&sl.acc[0][0])[i] = 0.f;
+      for (int extra = C::kNW - n_pairs; extra > 0; --extra) {  // largest cost per warp first
+        int best = 0;
+        for (int k = 1; k < n_pairs; ++k)
+          if ((long)cost[k] * wk[best] > (long)cost[best] * wk[k]) best = k;
+        ++wk[best];
+      }
+      int ww = 0;
+      for (int k = 0; k < n_pairs; ++k)
+        for (int j = 0; j < wk[k]; ++j, ++ww) s_warp_seg[ww] = k | ((k + 1) << 16);
+    } else {
+      for (int ww = 0; ww < C::kNW; ++ww)
+        s_warp_seg[ww] = (ww * n_pairs / C::kNW) | (((ww + 1) * n_pairs / C::kNW) << 16);
     }
-    if (threadIdx.x == 0) *s_ctr = it_begin;
   }
+  int seg_cur = 0, seg_hi = 0;  // this warp's segments, read after the barrier below
+  const int NG = sp.NG, S = args.S;
+  const long rec_stride = C::kRec;
+  // claims the next item of this warp's segments (warp-uniform; -1 when done)
+  auto claim = [&]() -> int {
+    while (seg_cur < seg_hi) {
+      int it = 0;
+      if (lane == 0) it = atomicAdd(&s_seg_next[seg_cur], 1);
+      it = __shfl_sync(0xffffffffu, it, 0);
+      if (it < s_seg_end[seg_cur]) return it;
+      ++seg_cur;
+    }
+    return -1;
+  };
+  // starts the copies of item `it` into item slot k: records from lane 0, the
+  // rows of a residual item from one lane each (row t of K: lane t, of V: lane 8 + t)
+  auto issue = [&](int it, int k) {
+    if (it < 0) return;
+    unsigned char* dst = wbase + k * C::kItemBytes;
+    const int pair = pair_of(sp, it), kk = it - pair * sp.ipp;
+    if (kk < sp.n2 + sp.n1) {
+      if (lane == 0) {
+        const int g0 = 2 * kk;
+        const int n_rec = kk < sp.n2 ? 2 : 1;
+        const uint32_t bytes = n_rec * C::kRec;
+#ifdef KIVI_DEBUG_BOUNDS
+        if (pair >= sp.pairs || g0 + n_rec > min(NG, args.ngcap)) {
+          atomicOr(args.status, kStatusBounds);
+          return;
+        }
+#endif
+        mbar_expect_tx(&bars[k], bytes + debug_overstate());
+        bulk_load(dst, args.records + ((long)pair * args.ngcap + g0) * rec_stride, bytes, &bars[k]);
+      }
+    } else {
+      const int t0 = NG * kGroup + kResTok * (kk - sp.n2 - sp.n1);
+      const int n = min(kResTok, S - t0);
+      const long row0 = (long)pair * kRingSlots + t0 % kRingSlots;
+#ifdef KIVI_DEBUG_BOUNDS
+      if (pair >= sp.pairs || n < 1 || t0 % kRingSlots + n > kRingSlots) {
+        if (lane == 0) atomicOr(args.status, kStatusBounds);
+        return;
+      }
+#endif
+      if (lane == 0) mbar_expect_tx(&bars[k], 2u * n * D * 2 + debug_overstate());
+      __syncwarp();
+      const int t = lane & 7;
+      if (lane < 16 && t < n) {
+        const bool v = lane >= 8;
+        bulk_load(dst + (v ? C::kRec : 0) + t * C::kResRow,
+                  (v ? args.ring_v : args.ring_k) + (row0 + t) * D, D * 2, &bars[k]);
+      }
+    }
+  };
+
   wait_for_predecessor();  // q, the records and the rings may come from the previous kernel
-  for (int k = warp; k < n_pairs; k += C::kNW) {
-    const int pair = p_first + k;
-    const int b = pair / args.Hkv, kvh = pair % args.Hkv;
-    const uint4* src =
-        reinterpret_cast<const uint4*>(args.q + ((long)b * args.Hq + (long)kvh * HPK) * D);
-    uint4* dst = reinterpret_cast<uint4*>(&slots[k].q[0][0]);
-    for (int i = lane; i < HPK * D / 8; i += 32) dst[i] = src[i];
+  __syncthreads();         // counters, segment table and mbarriers are set up
+  seg_cur = s_warp_seg[warp] & 0xffff;
+  seg_hi = s_warp_seg[warp] >> 16;
+  int itm[C::kItemSlots];
+#pragma unroll
+  for (int k = 0; k < C::kItemSlots; ++k) {
+    itm[k] = claim();
+    issue(itm[k], k);
   }
-  __syncthreads();
 
   const float qscale = (args.sm_scale > 0.f ? args.sm_scale : rsqrtf((float)D)) * kLog2e;
   W w(args, lane, qscale);
-  w.p_tile = wbase + 2 * C::kItemBytes;
+  w.p_tile = wbase + C::kItemSlots * C::kItemBytes;
   {
     const int hcol = w.g & 3;
     const bool lo_lane = C::kLoCols && w.g >= 4;
@@ -890,49 +999,8 @@ decode_kernel(DecodeArgs args, Split sp) {
   }
   w.reset();
 
-  const int NG = sp.NG, S = args.S;
-  const long rec_stride = C::kRec;
-  // claims the next item (warp-uniform result; -1 when the CTA's range is done)
-  auto claim = [&]() -> int {
-    int it = 0;
-    if (lane == 0) it = atomicAdd(s_ctr, 1);
-    it = __shfl_sync(0xffffffffu, it, 0);
-    return it < it_end ? it : -1;
-  };
-  // lane 0 starts the copies of item `it` into item slot k
-  auto issue = [&](int it, int k) {
-    if (lane != 0 || it < 0) return;
-    unsigned char* dst = wbase + k * C::kItemBytes;
-    const int pair = it / sp.ipp, kk = it % sp.ipp;
-    if (kk < sp.n2 + sp.n1) {
-      const int g0 = 2 * kk;
-      const uint32_t bytes = (kk < sp.n2 ? 2 : 1) * C::kRec;
-      mbar_expect_tx(&bars[k], bytes);
-      bulk_load(dst, args.records + ((long)pair * args.ngcap + g0) * rec_stride, bytes, &bars[k]);
-    } else {
-      const int t0 = NG * kGroup + kResTok * (kk - sp.n2 - sp.n1);
-      const int n = min(kResTok, S - t0);
-      const long row0 = (long)pair * kRingSlots + t0 % kRingSlots;
-      mbar_expect_tx(&bars[k], 2u * n * D * 2);
-      for (int t = 0; t < n; ++t) {
-        bulk_load(dst + t * C::kResRow, args.ring_k + (row0 + t) * D, D * 2, &bars[k]);
-        bulk_load(dst + C::kRec + t * C::kResRow, args.ring_v + (row0 + t) * D, D * 2, &bars[k]);
-      }
-    }
-  };
-
-  int itm[2];
-  itm[0] = claim();
-  issue(itm[0], 0);
-  itm[1] = claim();
-  issue(itm[1], 1);
-  int cur_pair = -1;
-  bool timed_out = false;
-  int i_stop = 0;
-
-  // merges this warp's state for `pair` into the CTA's slot
-  auto flush = [&](int pair) {
-    Slot& sl = slots[pair - p_first];
+  // this warp's state as m[HPK], l[HPK], acc[HPK][D] (fp32) at dst
+  auto export_state = [&](float* dst) {
     float lw[C::kChunks];
 #pragma unroll
     for (int c = 0; c < C::kChunks; ++c) {
@@ -942,132 +1010,68 @@ decode_kernel(DecodeArgs args, Split sp) {
       l += __shfl_xor_sync(0xffffffffu, l, 16);
       lw[c] = l;
     }
-    // final accumulators: (hi - lo') for <= 4 heads, times 2^shift, plus the value-min term
-    float F[W::kMTiles][4];
+    // accumulators: (hi - lo') for <= 4 heads, times 2^shift, plus the value-min term
     float vm[4];
 #pragma unroll
     for (int r = 0; r < 4; ++r) vm[r] = w.vmacc[r];
-#pragma unroll
-    for (int mt = 0; mt < W::kMTiles; ++mt)
-#pragma unroll
-      for (int r = 0; r < 4; ++r) F[mt][r] = w.acc[mt][r];
     if constexpr (C::kLoCols) {
-#pragma unroll
-      for (int mt = 0; mt < W::kMTiles; ++mt)
-#pragma unroll
-        for (int r = 0; r < 4; ++r) F[mt][r] -= __shfl_xor_sync(0xffffffffu, F[mt][r], 2);
 #pragma unroll
       for (int r = 0; r < 4; ++r) vm[r] -= __shfl_xor_sync(0xffffffffu, vm[r], 2);
     }
-#pragma unroll
-    for (int mt = 0; mt < W::kMTiles; ++mt)
-#pragma unroll
-      for (int r = 0; r < 4; ++r) F[mt][r] *= (float)(1 << C::kCodeShift);
-    // value-min term of block j, columns 2tig + e, sits in lane 4j + tig (rows g = j)
+    float vb[W::kBlocks][2];  // value-min term of block j, columns 2tig + e: lane 4j + tig
 #pragma unroll
     for (int j = 0; j < W::kBlocks; ++j) {
-      const float v0 = __shfl_sync(0xffffffffu, vm[0], 4 * j + w.tig);
-      const float v1 = __shfl_sync(0xffffffffu, vm[1], 4 * j + w.tig);
-#pragma unroll
-      for (int mi = 0; mi < 2; ++mi) {
-        F[2 * j + mi][0] += v0;
-        F[2 * j + mi][2] += v0;
-        F[2 * j + mi][1] += v1;
-        F[2 * j + mi][3] += v1;
-      }
+      vb[j][0] = __shfl_sync(0xffffffffu, vm[0], 4 * j + w.tig);
+      vb[j][1] = __shfl_sync(0xffffffffu, vm[1], 4 * j + w.tig);
     }
-    float Mw[2], Lw[2];
-    {
-      float mh[2], lh[2];
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int h = 2 * w.tig + e;  // head of accumulator column 2tig + e (hi lanes)
-        const int src = (lane & ~3) | (h & 3);
-        float m0 = __shfl_sync(0xffffffffu, w.m_run[0], src);
-        float l0 = __shfl_sync(0xffffffffu, lw[0], src);
-        if constexpr (C::kChunks == 2) {
-          const float m1 = __shfl_sync(0xffffffffu, w.m_run[C::kChunks - 1], src);
-          const float l1 = __shfl_sync(0xffffffffu, lw[C::kChunks - 1], src);
-          m0 = h >= 4 ? m1 : m0;
-          l0 = h >= 4 ? l1 : l0;
-        }
-        mh[e] = m0;
-        lh[e] = l0;
-      }
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        Mw[e] = mh[e];
-        Lw[e] = lh[e];
-      }
-    }
-    // lock the slot (bounded)
-    bool locked = true;
-    if (lane == 0) {
-      int spins = 0;
-      while (atomicCAS(&sl.lock, 0, 1) != 0) {
-        if (++spins > kLockSpinLimit) {
-          locked = false;
-          atomicOr(args.status, kStatusLockTimeout);
-          break;
-        }
-        __nanosleep(64);
-      }
-    }
-    locked = __shfl_sync(0xffffffffu, locked, 0);
-    if (!locked) return;
-    __threadfence_block();
     const bool valid_lane = C::kLoCols ? w.tig < 2 : true;
-    float newM[2], newL[2];
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int h = 2 * w.tig + e;
-      const bool valid = valid_lane && h < HPK;
-      const float Ms = sl.m[h & 7], Ls = sl.l[h & 7];
-      const float M = fmaxf(Ms, Mw[e]);
-      const float fs = Ms == -INFINITY ? 0.f : exp2f(Ms - M);
-      const float fw = Mw[e] == -INFINITY ? 0.f : exp2f(Mw[e] - M);
-      newM[e] = M;
-      newL[e] = Ls * fs + Lw[e] * fw;
-      if (valid) {
-        float* ah = sl.acc[h < HPK ? h : 0];
+    for (int mt = 0; mt < W::kMTiles; ++mt) {
 #pragma unroll
-        for (int mt = 0; mt < W::kMTiles; ++mt) {
-          ah[16 * mt + w.g] = ah[16 * mt + w.g] * fs + F[mt][e] * fw;
-          ah[16 * mt + w.g + 8] = ah[16 * mt + w.g + 8] * fs + F[mt][e + 2] * fw;
-        }
+      for (int r = 0; r < 4; ++r) {
+        float x = w.acc[mt][r];
+        if constexpr (C::kLoCols) x -= __shfl_xor_sync(0xffffffffu, x, 2);
+        x = x * (float)(1 << C::kCodeShift) + vb[mt / 2][r & 1];
+        const int h = 2 * w.tig + (r & 1);
+        if (valid_lane && h < HPK) dst[2 * HPK + h * D + 16 * mt + w.g + 8 * (r >> 1)] = x;
       }
     }
-    __syncwarp();
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int h = 2 * w.tig + e;
-      if (valid_lane && h < HPK && w.g == 0) {
-        sl.m[h] = newM[e];
-        sl.l[h] = newL[e];
+    for (int c = 0; c < C::kChunks; ++c) {
+      const int h = 4 * c + w.tig;
+      if (w.g == 0 && h < HPK) {
+        dst[h] = w.m_run[c];
+        dst[HPK + h] = lw[c];
       }
     }
-    __threadfence_block();
-    __syncwarp();
-    if (lane == 0) atomicExch(&sl.lock, 0);
   };
 
+  int cur_pair = -1;
+  bool timed_out = false;
+  int i_stop = 0;
+  const long park_stride = park_stride_floats(D, HPK);
+
   for (int i = 0;; ++i) {
-    const int k = i & 1;
+    const int k = i % C::kItemSlots;
     const int it = itm[k];
     if (it < 0) break;
-    const bool arrived = mbar_wait_bounded(&bars[k], (uint32_t)(i >> 1) & 1u);
+    const bool arrived = mbar_wait_bounded(&bars[k], (uint32_t)(i / C::kItemSlots) & 1u);
     if (!__all_sync(0xffffffffu, arrived)) {
       timed_out = true;
       i_stop = i;
       break;
     }
-    const int pair = it / sp.ipp, kk = it % sp.ipp;
+    const int pair = pair_of(sp, it), kk = it - pair * sp.ipp;
     if (pair != cur_pair) {
       if (cur_pair >= 0) {
-        flush(cur_pair);
+        // park the state of the pair this warp leaves: its own slot, no lock
+        export_state(args.parks + ((long)cur_pair * kParkWarps + warp) * park_stride);
+        if (lane == 0) atomicOr(&s_parked[cur_pair - p_first], 1u << warp);
         w.reset();
       }
-      w.load_pair(&slots[pair - p_first].q[0][0]);
+      // the pair's q (global, HPK x D bf16): read by the warp itself, so its
+      // latency hides under the first item's copy
+      w.load_pair(args.q + ((long)(pair / args.Hkv) * args.Hq + (long)(pair % args.Hkv) * HPK) * D);
       cur_pair = pair;
     }
     unsigned char* base = wbase + k * C::kItemBytes;
@@ -1085,77 +1089,157 @@ decode_kernel(DecodeArgs args, Split sp) {
   }
   if (timed_out) {
     // record the failure, then give the copies still in flight a bounded chance
-    // to land before this CTA's shared memory is released
+    // to land before this CTA's shared memory is reused
     if (lane == 0) {
       atomicOr(args.status, kStatusWaitTimeout);
-      for (int j = i_stop; j < i_stop + 2; ++j)
-        if (itm[j & 1] >= 0) (void)mbar_wait_bounded(&bars[j & 1], (uint32_t)(j >> 1) & 1u);
+      for (int j = i_stop; j < i_stop + C::kItemSlots; ++j)
+        if (itm[j % C::kItemSlots] >= 0)
+          (void)mbar_wait_bounded(&bars[j % C::kItemSlots], (uint32_t)(j / C::kItemSlots) & 1u);
     }
     __syncwarp();
   }
-  if (cur_pair >= 0) flush(cur_pair);
+  // the final state goes to this warp's own item slots (no copy is in flight any more)
+  if (cur_pair >= 0) {
+    export_state(reinterpret_cast<float*>(wbase));
+    if (lane == 0) s_final[warp] = cur_pair - p_first;
+  }
+  __threadfence_block();
   __syncthreads();
   allow_successor();
 
-  // ---- outputs: whole pairs directly, shared pairs through partials and tickets ----
-  constexpr int kPart = HPK * (D + 2);  // floats of one partial: m[HPK], l[HPK], acc[HPK][D]
-  for (int k = warp; k < n_pairs; k += C::kNW) {
-    const int pair = p_first + k;
-    const Slot& sl = slots[k];
+  // ---- merge the warps of each pair (all threads), then write the outputs ----
+  // Pairs held whole by this CTA go to `out`; a pair shared with other CTAs goes
+  // to this CTA's partial, and the last CTA to arrive merges the partials.
+  constexpr int kPart = HPK * (D + 2);  // floats of a partial: m[HPK], l[HPK], acc[HPK][D]
+  // merge tables over the (now unused) q slots, for a batch of pairs at once:
+  // the kind of each warp's state for pair k (0 none, 1 its final state in its
+  // own shared slots, 2 parked in global memory), its (m, l) and factor
+  // 2^(m - M) per head, the merged M and L, and where the result goes
+  const int nw = C::kNW;
+  constexpr int kTableBytes = C::kNW * 4 + C::kNW * HPK * 12 + HPK * 8 + 16;
+  constexpr int kBatch = C::kSlots * C::kSlotBytes / kTableBytes;
+  static_assert(kBatch >= 1, "merge tables of one pair fit the q slots");
+  bool wrote_partial = false;
+  for (int k0 = 0; k0 < n_pairs; k0 += kBatch) {
+    const int nb = min(kBatch, n_pairs - k0);
+    int* s_kind = reinterpret_cast<int*>(smem + C::kOffSlots);  // [nb][kNW]
+    float* s_m = reinterpret_cast<float*>(s_kind + nb * nw);      // [nb][kNW][HPK]
+    float* s_l = s_m + nb * nw * HPK;
+    float* s_f = s_l + nb * nw * HPK;
+    float* s_ML = s_f + nb * nw * HPK;                              // [nb][2][HPK]
+    int* s_dest = reinterpret_cast<int*>(s_ML + nb * 2 * HPK);      // [nb]: -1 out, else side
+    int* s_anypark = s_dest + nb;                                   // [nb]
+    for (int t = threadIdx.x; t < nb * nw; t += C::kThreads) {
+      const int k = k0 + t / nw, ww = t % nw;
+      s_kind[t] = s_final[ww] == k ? 1 : ((s_parked[k] >> ww & 1u) ? 2 : 0);
+    }
+    __syncthreads();
+    for (int t = threadIdx.x; t < nb * nw * HPK; t += C::kThreads) {  // every state header
+      const int kw = t / HPK, h = t % HPK, ww = kw % nw;
+      const int kind = s_kind[kw];
+      const float* src = kind == 1 ? reinterpret_cast<const float*>(smem + ww * C::kWarpBytes)
+                                   : args.parks + ((long)(p_first + k0 + kw / nw) * kParkWarps + ww) * park_stride;
+      s_m[t] = kind ? src[h] : -INFINITY;
+      s_l[t] = kind ? src[HPK + h] : 0.f;
+    }
+    __syncthreads();
+    for (int t = threadIdx.x; t < nb * HPK; t += C::kThreads) {
+      const int kb = t / HPK, h = t % HPK;
+      float M = -INFINITY;
+      for (int ww = 0; ww < nw; ++ww) M = fmaxf(M, s_m[(kb * nw + ww) * HPK + h]);
+      float L = 0.f;
+      for (int ww = 0; ww < nw; ++ww) {
+        const int i = (kb * nw + ww) * HPK + h;
+        const float f = s_m[i] == -INFINITY ? 0.f : exp2f(s_m[i] - M);
+        L += s_l[i] * f;
+        s_f[i] = f;
+      }
+      s_ML[kb * 2 * HPK + h] = M;
+      s_ML[kb * 2 * HPK + HPK + h] = L;
+      if (h == 0) {
+        const int pair = p_first + k0 + kb;
+        const int fc = cta_of_item(sp, pair * sp.ipp);
+        const int lc = cta_of_item(sp, pair * sp.ipp + sp.ipp - 1);
+        s_dest[kb] = fc == lc ? -1 : (pair == p_first ? 0 : 1);
+        int any = 0;
+        for (int ww = 0; ww < nw; ++ww) any |= s_kind[kb * nw + ww] == 2;
+        s_anypark[kb] = any;
+      }
+    }
+    __syncthreads();
+    for (int t = threadIdx.x; t < nb * HPK * D; t += C::kThreads) {
+      const int kb = t / (HPK * D), e = t % (HPK * D), h = e / D;
+      const int pair = p_first + k0 + kb;
+      const float* f = s_f + kb * nw * HPK + h;
+      float A = 0.f;
+#pragma unroll
+      for (int ww = 0; ww < C::kNW; ++ww)  // final states in the warps' own slots
+        if (s_kind[kb * nw + ww] == 1)
+          A = fmaf(f[ww * HPK], reinterpret_cast<const float*>(smem + ww * C::kWarpBytes)[2 * HPK + e], A);
+      if (s_anypark[kb]) {  // parked states (a warp that swept several segments)
+        for (int ww = 0; ww < nw; ++ww)
+          if (s_kind[kb * nw + ww] == 2)
+            A = fmaf(f[ww * HPK], args.parks[((long)pair * kParkWarps + ww) * park_stride + 2 * HPK + e], A);
+      }
+      const int dest = s_dest[kb];
+      if (dest < 0) {
+        const int b = pair / args.Hkv, kvh = pair % args.Hkv;
+        args.out[((long)b * args.Hq + (long)kvh * HPK) * D + e] = A / s_ML[kb * 2 * HPK + HPK + h];
+      } else if (cta < args.max_ctas) {
+        float* part = args.partials + ((long)cta * 2 + dest) * kPart;
+        part[2 * HPK + e] = A;
+        if (e % D == 0) {
+          part[h] = s_ML[kb * 2 * HPK + h];
+          part[HPK + h] = s_ML[kb * 2 * HPK + HPK + h];
+        }
+        wrote_partial = true;
+      }
+    }
+    __syncthreads();  // the tables are rebuilt for the next batch
+  }
+  if (__syncthreads_or(wrote_partial)) __threadfence();
+  // tickets of the shared pairs (only the first and the last pair of a CTA can
+  // be shared): thread 0 takes them; the CTA that arrives last at a pair merges
+  // that pair's partials with all its threads
+  int* s_last = reinterpret_cast<int*>(smem + C::kOffSlots);  // [2]: pair this CTA completes, or -1
+  if (threadIdx.x < 2) s_last[threadIdx.x] = -1;
+  __syncthreads();
+  if (threadIdx.x < 2 && cta < args.max_ctas) {  // both tickets at once
+    const int side = threadIdx.x;
+    const int pair = side == 0 ? p_first : p_last;
+    if (side == 0 || p_last != p_first) {
+      const int fc = cta_of_item(sp, pair * sp.ipp), lc = cta_of_item(sp, pair * sp.ipp + sp.ipp - 1);
+      if (fc != lc && atomicAdd(&args.tickets[pair], 1) == lc - fc) s_last[side] = pair;
+    }
+  }
+  if (threadIdx.x == 0 && cta >= args.max_ctas) atomicOr(args.status, kStatusBadSplit);
+  __syncthreads();
+  for (int side = 0; side < 2; ++side) {
+    const int pair = s_last[side];
+    if (pair < 0) continue;
+    __threadfence();
     const int fc = cta_of_item(sp, pair * sp.ipp), lc = cta_of_item(sp, pair * sp.ipp + sp.ipp - 1);
     const int b = pair / args.Hkv, kvh = pair % args.Hkv;
     float* out = args.out + ((long)b * args.Hq + (long)kvh * HPK) * D;
-    if (fc == lc) {
-      for (int i = lane; i < HPK * D; i += 32) out[i] = sl.acc[i / D][i % D] / sl.l[i / D];
-      continue;
-    }
-    const int side = pair == p_first ? 0 : 1;
-    if (cta >= args.max_ctas) {  // the host sizes the partials for every grid it launches
-      if (lane == 0) atomicOr(args.status, kStatusBadSplit);
-      continue;
-    }
-    float* part = args.partials + ((long)cta * 2 + side) * kPart;
-    if (lane < HPK) {
-      part[lane] = sl.m[lane];
-      part[HPK + lane] = sl.l[lane];
-    }
-    for (int i = lane; i < HPK * D; i += 32) part[2 * HPK + i] = sl.acc[i / D][i % D];
-    __threadfence();
-    __syncwarp();
-    int prev = 0;
-    if (lane == 0) prev = atomicAdd(&args.tickets[pair], 1);
-    prev = __shfl_sync(0xffffffffu, prev, 0);
-    if (prev != lc - fc) continue;
-    // the last CTA of this pair: merge the partials of CTAs fc..lc
-    __threadfence();
-    float M = -INFINITY, L = 0.f;
-    if (lane < HPK) {
+    // partial of CTA ct: side 0 if the pair is ct's first pair (only fc can hold
+    // it as its last pair)
+    for (int e = threadIdx.x; e < HPK * D; e += C::kThreads) {
+      const int h = e / D;
+      float M = -INFINITY, L = 0.f, A = 0.f;  // online merge: the loads of all parts overlap
+#pragma unroll 4
       for (int ct = fc; ct <= lc; ++ct) {
-        const int sd = (cta_first_item(sp, ct) / sp.ipp) == pair ? 0 : 1;
-        const float* pp = args.partials + ((long)ct * 2 + sd) * kPart;
-        M = fmaxf(M, __ldcg(pp + lane));
+        const float* pp = args.partials + ((long)ct * 2 + (ct == fc && pair != cta_first_item(sp, ct) / sp.ipp ? 1 : 0)) * kPart;
+        const float m = __ldcg(pp + h), l = __ldcg(pp + HPK + h), a = __ldcg(pp + 2 * HPK + e);
+        const float Mn = fmaxf(M, m);
+        const float fo = M == -INFINITY ? 0.f : exp2f(M - Mn), fn = exp2f(m - Mn);
+        L = L * fo + l * fn;
+        A = A * fo + a * fn;
+        M = Mn;
       }
-      for (int ct = fc; ct <= lc; ++ct) {
-        const int sd = (cta_first_item(sp, ct) / sp.ipp) == pair ? 0 : 1;
-        const float* pp = args.partials + ((long)ct * 2 + sd) * kPart;
-        L += __ldcg(pp + HPK + lane) * exp2f(__ldcg(pp + lane) - M);
-      }
+      out[e] = A / L;
     }
-    for (int i = lane; i < HPK * D; i += 32) {
-      const int h = i / D;
-      const float Mh = __shfl_sync(0xffffffffu, M, h);
-      const float Lh = __shfl_sync(0xffffffffu, L, h);
-      float o = 0.f;
-      for (int ct = fc; ct <= lc; ++ct) {
-        const int sd = (cta_first_item(sp, ct) / sp.ipp) == pair ? 0 : 1;
-        const float* pp = args.partials + ((long)ct * 2 + sd) * kPart;
-        o += exp2f(__ldcg(pp + h) - Mh) * __ldcg(pp + 2 * HPK + i);
-      }
-      out[i] = o / Lh;
-    }
-    if (lane == 0) args.tickets[pair] = 0;  // ready for the next call
+    if (threadIdx.x == 0) args.tickets[pair] = 0;  // ready for the next call
   }
-  (void)s_flag;
 }
 
 // ---------------------------------------------------------------------------
@@ -1173,6 +1257,8 @@ Split make_split(int pairs, int S, int num_sms) {
   s.n1 = s.NG % 2;
   s.nr = (r + kResTok - 1) / kResTok;
   s.ipp = s.n2 + s.n1 + s.nr;
+  // ceil(2^64 / ipp) = floor((2^64 - 1) / ipp) + 1 for ipp >= 2
+  if (s.ipp >= 2) s.ipp_inv = ~0ULL / (unsigned long long)s.ipp + 1;
   s.c2 = C::kCostG2;
   s.c1 = C::kCostG1;
   s.cr = C::kCostR;
@@ -1258,6 +1344,15 @@ int pair_slots(int D, int bits, int hpk) {
 
 }  // namespace
 
+cudaError_t debug_overstate_copies(unsigned bytes) {
+#ifdef KIVI_DEBUG_BUILD
+  return cudaMemcpyToSymbol(g_kivi_debug_overstate, &bytes, sizeof bytes);
+#else
+  (void)bytes;
+  return cudaErrorNotSupported;
+#endif
+}
+
 int decode_max_ctas(int D, int bits, int hpk, long pairs) {
   const int slots = pair_slots(D, bits, hpk);
   if (slots < 2) return 0;
@@ -1275,9 +1370,16 @@ int decode_grid_ctas(int D, int bits, int hpk, long pairs, int S, int num_sms) {
   return 0;
 }
 
+long decode_parks_bytes(int D, int hpk, long pairs) {
+  return pairs * kParkWarps * park_stride_floats(D, hpk) * (long)sizeof(float);
+}
+
+long decode_partial_bytes(int D, int hpk) { return 2L * hpk * (D + 2) * (long)sizeof(float); }
+
 long decode_workspace_bytes(int D, int bits, int hpk, long pairs) {
   const long ctas = decode_max_ctas(D, bits, hpk, pairs);
-  return kWsHeader + ws_tickets_bytes(pairs) + ctas * 2L * hpk * (D + 2) * (long)sizeof(float);
+  return kWsHeader + ws_tickets_bytes(pairs) + decode_parks_bytes(D, hpk, pairs) +
+         ctas * decode_partial_bytes(D, hpk);
 }
 
 cudaError_t launch_decode(int D, int bits, const DecodeArgs& a, cudaStream_t stream) {

@@ -35,6 +35,7 @@ struct DecodeArgs {
   float* out;                    // [B][Hq][D]
   uint32_t* status;              // device status word
   int* tickets;                  // one per (sequence, kv head); zero between calls
+  float* parks;                  // [B*Hkv][16 warps] parked warp states
   float* partials;               // [max_ctas][2][Hq/Hkv][D + 2] split partials
   int max_ctas;                  // capacity of `partials` in CTAs
   int B, Hkv, Hq, S, ngcap;
@@ -43,14 +44,21 @@ struct DecodeArgs {
   int device;                    // the CUDA device the buffers live on (current at launch)
 };
 
-// Largest grid the decode kernel uses for `pairs` (sequence, kv head) pairs,
-// and the workspace bytes (status header, tickets, partials) that grid needs.
-// Host-only arithmetic; no device is queried.
+// Workspace of the decode kernel for `pairs` (sequence, kv head) pairs, in
+// order: status header, tickets, parked warp states (parks_bytes), then the
+// per-CTA partials (partial_bytes each) of the largest grid it uses
+// (decode_max_ctas).  Host-only arithmetic; no device is queried.
 int decode_max_ctas(int D, int bits, int hpk, long pairs);
+long decode_parks_bytes(int D, int hpk, long pairs);
+long decode_partial_bytes(int D, int hpk);
 // CTAs the decode kernel launches for this shape on a device with num_sms SMs
 // (0 for an unsupported shape).
 int decode_grid_ctas(int D, int bits, int hpk, long pairs, int S, int num_sms);
 long decode_workspace_bytes(int D, int bits, int hpk, long pairs);
+
+// Debug build only (KIVI_DEBUG_BUILD): bytes added to every expected copy size
+// of the decode kernel; cudaErrorNotSupported in a regular build.
+cudaError_t debug_overstate_copies(unsigned bytes);
 
 cudaError_t launch_prefill(int D, int bits, const PrefillArgs& a, cudaStream_t stream);
 cudaError_t launch_append(int D, int bits, const AppendArgs& a, cudaStream_t stream);

@@ -11,9 +11,11 @@ from .oracle import (  # noqa: F401
     R,
     OracleCache,
     attend_one,
+    attention_bf16,
     cache_bytes,
     dequant_record,
     f16_bits_to_double,
+    fake_quant_keys,
     f32_to_f16_bits,
     make_record,
     num_groups,

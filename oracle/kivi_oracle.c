@@ -360,28 +360,11 @@ int oracle_append(const uint16_t* k_new, const uint16_t* v_new, int B, int Hkv, 
   return S + 1;
 }
 
-/* Decode attention of one query head over one kv head holding S tokens:
- * scores s_t = sm_scale * <q, k_hat_t>, out = sum_t softmax(s)_t v_hat_t, in
- * double.  k_hat/v_hat are the dequantized groups for t < NG*G and the bf16
- * residual otherwise. */
-void oracle_attend_one(const uint8_t* seq_records, const uint16_t* seq_ring_k,
-                       const uint16_t* seq_ring_v, const uint16_t* q, int S, int D,
-                       int bits, double sm_scale, double* out) {
-  const int G = ORACLE_G, slots = ORACLE_R + ORACLE_G;
-  const int NG = oracle_num_groups(S);
-  const long rb = oracle_record_bytes(D, bits);
-  double* K = (double*)malloc(sizeof(double) * (size_t)S * D);
-  double* V = (double*)malloc(sizeof(double) * (size_t)S * D);
+/* Softmax attention of one query row over S dense (K, V) rows [S][D] in
+ * double: s_t = sm_scale * <q, k_t>, out = sum_t softmax(s)_t v_t. */
+static void attend_dense(const double* K, const double* V, const uint16_t* q, int S, int D,
+                         double sm_scale, double* out) {
   double* s = (double*)malloc(sizeof(double) * (size_t)(S > 0 ? S : 1));
-  for (int g = 0; g < NG; ++g)
-    oracle_dequant_record(seq_records + g * rb, D, bits, K + (long)g * G * D,
-                          V + (long)g * G * D);
-  for (int t = NG * G; t < S; ++t) {
-    for (int d = 0; d < D; ++d) {
-      K[(long)t * D + d] = bf16_bits_to_float(seq_ring_k[(long)(t % slots) * D + d]);
-      V[(long)t * D + d] = bf16_bits_to_float(seq_ring_v[(long)(t % slots) * D + d]);
-    }
-  }
   double m = -INFINITY;
   for (int t = 0; t < S; ++t) {
     double acc = 0.0;
@@ -399,9 +382,33 @@ void oracle_attend_one(const uint8_t* seq_records, const uint16_t* seq_ring_k,
     for (int t = 0; t < S; ++t) acc += s[t] * V[(long)t * D + d];
     out[d] = acc / denom;
   }
+  free(s);
+}
+
+/* Decode attention of one query head over one kv head holding S tokens:
+ * scores s_t = sm_scale * <q, k_hat_t>, out = sum_t softmax(s)_t v_hat_t, in
+ * double.  k_hat/v_hat are the dequantized groups for t < NG*G and the bf16
+ * residual otherwise. */
+void oracle_attend_one(const uint8_t* seq_records, const uint16_t* seq_ring_k,
+                       const uint16_t* seq_ring_v, const uint16_t* q, int S, int D,
+                       int bits, double sm_scale, double* out) {
+  const int G = ORACLE_G, slots = ORACLE_R + ORACLE_G;
+  const int NG = oracle_num_groups(S);
+  const long rb = oracle_record_bytes(D, bits);
+  double* K = (double*)malloc(sizeof(double) * (size_t)(S > 0 ? S : 1) * D);
+  double* V = (double*)malloc(sizeof(double) * (size_t)(S > 0 ? S : 1) * D);
+  for (int g = 0; g < NG; ++g)
+    oracle_dequant_record(seq_records + g * rb, D, bits, K + (long)g * G * D,
+                          V + (long)g * G * D);
+  for (int t = NG * G; t < S; ++t) {
+    for (int d = 0; d < D; ++d) {
+      K[(long)t * D + d] = bf16_bits_to_float(seq_ring_k[(long)(t % slots) * D + d]);
+      V[(long)t * D + d] = bf16_bits_to_float(seq_ring_v[(long)(t % slots) * D + d]);
+    }
+  }
+  attend_dense(K, V, q, S, D, sm_scale, out);
   free(K);
   free(V);
-  free(s);
 }
 
 /* Decode attention of a whole layer: q [B][Hq][D] bf16 -> out [B][Hq][D]
@@ -419,5 +426,74 @@ void oracle_attention(const uint8_t* records, const uint16_t* ring_k,
                         ring_v + seq * slots * D, q + ((long)b * Hq + h) * D, S, D, bits,
                         sm_scale, out + ((long)b * Hq + h) * D);
     }
+  }
+}
+
+/* ------------------------------------------------------------------------ */
+/* The full-precision baseline: attention over an unquantized bf16 cache    */
+/* ------------------------------------------------------------------------ */
+
+/* Decode attention over a bf16 cache, the 16-bit baseline the [HF page] and
+ * the [KIVI page] compare the quantized cache with.  k, v: bf16 bits
+ * [B][Hkv][Smax][D], tokens 0..S-1 of each (sequence, kv head) used; q: bf16
+ * bits [B][Hq][D]; out: [B][Hq][D] double.  Query head h reads kv head
+ * h / (Hq / Hkv). */
+void oracle_attention_bf16(const uint16_t* k, const uint16_t* v, const uint16_t* q, int B,
+                           int Hkv, int Hq, int S, int Smax, int D, double sm_scale,
+                           double* out) {
+  const int per_kv = Hq / Hkv;
+  double* K = (double*)malloc(sizeof(double) * (size_t)(S > 0 ? S : 1) * D);
+  double* V = (double*)malloc(sizeof(double) * (size_t)(S > 0 ? S : 1) * D);
+  for (int b = 0; b < B; ++b) {
+    for (int kvh = 0; kvh < Hkv; ++kvh) {
+      const long base = ((long)b * Hkv + kvh) * Smax * D;
+      for (long i = 0; i < (long)S * D; ++i) {
+        K[i] = bf16_bits_to_float(k[base + i]);
+        V[i] = bf16_bits_to_float(v[base + i]);
+      }
+      for (int j = 0; j < per_kv; ++j) {
+        const long row = (long)b * Hq + (long)kvh * per_kv + j;
+        attend_dense(K, V, q + row * D, S, D, sm_scale, out + row * D);
+      }
+    }
+  }
+  free(K);
+  free(V);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Key-granularity ablation: fake quantization of a key tile                */
+/* ------------------------------------------------------------------------ */
+
+/* Quantizes and dequantizes keys k (bf16 bits [T][D], T a multiple of G) with
+ * b bits, returning k_hat [T][D] in double:
+ *   per_token == 0: KIVI's key quantization ([KIVI page], [HF page]): each
+ *     channel of each G-token group is one group (the group record's keys);
+ *   per_token != 0: the granularity the pages argue against for keys: each
+ *     token's channels in blocks of G form one group (the values' rule).
+ * Parameters and codes follow the same quantizer and fp16 metadata as the
+ * record; k_hat = f16(scale) * code + f16(min). */
+void oracle_fake_quant_keys(const uint16_t* k, int T, int D, int bits, int per_token,
+                            double* k_hat) {
+  const int G = ORACLE_G;
+  /* group n (n_groups of G elements each): element i sits at k[first + i * step] */
+  const long n_groups = per_token ? (long)T * (D / G) : (long)(T / G) * D;
+  for (long n = 0; n < n_groups; ++n) {
+    long first, step;
+    if (per_token) {  /* token n / (D/G), channels G * (n % (D/G)) .. + G-1 */
+      first = (n / (D / G)) * D + (long)G * (n % (D / G));
+      step = 1;
+    } else {          /* channel n % D of tokens G * (n / D) .. + G-1 */
+      first = (n / D) * G * D + n % D;
+      step = D;
+    }
+    float x[ORACLE_G];
+    uint8_t codes[ORACLE_G];
+    for (int i = 0; i < G; ++i) x[i] = bf16_bits_to_float(k[first + i * step]);
+    float scale, mn;
+    oracle_quantize_group(x, G, 1, bits, &scale, &mn, codes);
+    const double sh = oracle_f16_bits_to_double(oracle_f32_to_f16_bits(scale));
+    const double mh = oracle_f16_bits_to_double(oracle_f32_to_f16_bits(mn));
+    for (int i = 0; i < G; ++i) k_hat[first + i * step] = sh * codes[i] + mh;
   }
 }

@@ -78,6 +78,10 @@ def _c():
         lib.oracle_attend_one.restype = None
         lib.oracle_attention.argtypes = [u8p, u16p, u16p, u16p, i, i, i, i, i, i, i, d, f64p]
         lib.oracle_attention.restype = None
+        lib.oracle_attention_bf16.argtypes = [u16p, u16p, u16p, i, i, i, i, i, i, d, f64p]
+        lib.oracle_attention_bf16.restype = None
+        lib.oracle_fake_quant_keys.argtypes = [u16p, i, i, i, i, f64p]
+        lib.oracle_fake_quant_keys.restype = None
         _lib = lib
     return _lib
 
@@ -152,6 +156,44 @@ def attend_one(seq_records, seq_ring_k, seq_ring_v, q_row, S, bits, sm_scale):
                            _p(seq_ring_v, ctypes.c_uint16),
                            _p(np.ascontiguousarray(q_row, np.uint16), ctypes.c_uint16),
                            S, D, bits, float(sm_scale), _p(out, ctypes.c_double))
+    return out
+
+
+def attention_bf16(k: np.ndarray, v: np.ndarray, q: np.ndarray, S: int | None = None,
+                   sm_scale: float | None = None) -> np.ndarray:
+    """Decode attention over an unquantized bf16 cache (the 16-bit baseline).
+
+    k, v: bf16 bits [B][Hkv][Smax][D] (tokens 0..S-1 used); q: bf16 bits [B][Hq][D]
+    -> float64 [B][Hq][D]; query head h reads kv head h // (Hq // Hkv).
+    """
+    k = np.ascontiguousarray(k, np.uint16)
+    v = np.ascontiguousarray(v, np.uint16)
+    q = np.ascontiguousarray(q, np.uint16)
+    B, Hkv, Smax, D = k.shape
+    Hq = q.shape[1]
+    assert Hq % Hkv == 0 and q.shape == (B, Hq, D)
+    S = Smax if S is None else S
+    scale = 1.0 / math.sqrt(D) if sm_scale is None or sm_scale <= 0 else float(sm_scale)
+    out = np.zeros((B, Hq, D), np.float64)
+    _c().oracle_attention_bf16(_p(k, ctypes.c_uint16), _p(v, ctypes.c_uint16),
+                               _p(q, ctypes.c_uint16), B, Hkv, Hq, S, Smax, D, scale,
+                               _p(out, ctypes.c_double))
+    return out
+
+
+def fake_quant_keys(k: np.ndarray, bits: int, per_token: bool) -> np.ndarray:
+    """Quantize-dequantize keys (bf16 bits [T][D], T a multiple of G) -> float64.
+
+    per_token=False: per channel over G-token groups (KIVI's key rule);
+    per_token=True: per token over G-channel blocks (the values' rule applied to
+    keys, the granularity the [KIVI page] and the [HF page] argue against).
+    """
+    k = np.ascontiguousarray(k, np.uint16)
+    T, D = k.shape
+    assert T % G == 0 and D % G == 0
+    out = np.zeros((T, D), np.float64)
+    _c().oracle_fake_quant_keys(_p(k, ctypes.c_uint16), T, D, bits, int(per_token),
+                                _p(out, ctypes.c_double))
     return out
 
 

@@ -20,8 +20,8 @@ def lib():
     return N.lib()
 
 
-def _header_functions():
-    text = open(os.path.join(ROOT, "include", "kivi.h")).read()
+def _header_functions(header="kivi.h"):
+    text = open(os.path.join(ROOT, "include", header)).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(kivi_[a-z_]+)\s*\(", text)))
 
@@ -31,6 +31,16 @@ def test_exports_every_declared_symbol(lib):
     assert len(names) >= 11
     for n in names:
         assert hasattr(lib, n), n
+
+
+def test_debug_library_exports_its_header():
+    """libkivi_debug.so exports the regular ABI plus the debug header's hook; the
+    regular library does not carry the hook."""
+    dbg = ctypes.CDLL(B.build(debug=True))
+    for n in _header_functions() + _header_functions("kivi_debug.h"):
+        assert hasattr(dbg, n), n
+    assert _header_functions("kivi_debug.h") == ["kivi_debug_overstate_copies"]
+    assert not hasattr(ctypes.CDLL(B.build()), "kivi_debug_overstate_copies")
 
 
 def cfg(**kw):

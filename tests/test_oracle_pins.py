@@ -417,3 +417,88 @@ def test_per_channel_keys_beat_per_token_on_outlier_channels():
             s, m, c = O.quantize_group(kf[t, j:j + 32], 2)
             err_t += np.abs(kf[t, j:j + 32] - (s * c + m)).sum()
     assert err_c < err_t
+
+
+# ---------------------------------------------------------------------------
+# The 16-bit baseline: attention over an unquantized bf16 cache
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("B,Hkv,Hq,S,Smax,D", [(2, 2, 8, 77, 80, 64), (1, 3, 3, 1, 4, 128),
+                                               (2, 1, 4, 300, 300, 128)])
+def test_bf16_attention_equals_library_sdpa(B, Hkv, Hq, S, Smax, D):
+    """Unused capacity (tokens S..Smax-1) holds NaN and must not reach the result."""
+    rng = np.random.default_rng(S + D)
+    k = torch.tensor(rng.standard_normal((B, Hkv, Smax, D))).to(torch.bfloat16)
+    v = torch.tensor(rng.standard_normal((B, Hkv, Smax, D))).to(torch.bfloat16)
+    k[:, :, S:] = float("nan")
+    v[:, :, S:] = float("nan")
+    q = torch.tensor(rng.standard_normal((B, Hq, D))).to(torch.bfloat16)
+    out = O.attention_bf16(_bits(k), _bits(v), _bits(q), S)
+    np.testing.assert_allclose(out, _sdpa(q, k[:, :, :S], v[:, :, :S], 1 / math.sqrt(D)),
+                               rtol=0, atol=1e-12)
+
+
+def test_bf16_attention_hand_worked():
+    g = _golden("hand_worked.json")["attention"]
+    D = 32
+    k = torch.zeros(1, 1, 2, D)
+    v = torch.zeros(1, 1, 2, D)
+    q = torch.zeros(1, 1, D)
+    q[0, 0, 0] = k[0, 0, 0, 0] = v[0, 0, 0, 0] = v[0, 0, 1, 1] = 1
+    out = O.attention_bf16(_bits(k), _bits(v), _bits(q), sm_scale=1.0)
+    assert out[0, 0, 0] == pytest.approx(g["out0"], abs=1e-15)
+    assert out[0, 0, 1] == pytest.approx(g["out1"], abs=1e-15)
+    assert np.all(out[0, 0, 2:] == 0)
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_bf16_attention_equals_quantized_cache_on_grid_inputs(bits):
+    """On grid inputs the quantized cache dequantizes exactly, so the two oracles,
+    which share only the final softmax loop, must agree."""
+    rng = np.random.default_rng(40 + bits)
+    B, Hkv, Hq, D, S = 1, 2, 4, 64, 290
+    n_q = O.num_groups(S) * O.G
+    k = torch.tensor(rng.standard_normal((B, Hkv, S, D)), dtype=torch.float64)
+    v = torch.tensor(rng.standard_normal((B, Hkv, S, D)), dtype=torch.float64)
+    for h in range(Hkv):
+        k[0, h, :n_q] = _grid_tile(rng, n_q, D, bits, "k")
+        v[0, h, :n_q] = _grid_tile(rng, n_q, D, bits, "v")
+    k, v = k.to(torch.bfloat16), v.to(torch.bfloat16)
+    q = torch.tensor(rng.standard_normal((B, Hq, D)) * 0.3).to(torch.bfloat16)
+    c = O.OracleCache(B, Hkv, D, bits, S)
+    c.prefill(_bits(k), _bits(v))
+    np.testing.assert_allclose(O.attention_bf16(_bits(k), _bits(v), _bits(q)),
+                               c.attention(_bits(q)), rtol=0, atol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# Key-granularity ablation: per channel (KIVI) against per token
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_fake_quant_keys_matches_the_record_paths(bits):
+    """Per channel is the record's key path; per token is the record's value path
+    applied to the keys (both packed, stored and read back by the record code)."""
+    rng = np.random.default_rng(bits)
+    D = 128
+    k = torch.tensor(rng.standard_normal((64, D)) * np.exp(rng.standard_normal(D))).to(
+        torch.bfloat16)
+    kb = _bits(k)
+    per_c = O.fake_quant_keys(kb, bits, per_token=False)
+    per_t = O.fake_quant_keys(kb, bits, per_token=True)
+    for g0 in (0, 32):
+        rec = O.make_record(kb[g0:g0 + 32], kb[g0:g0 + 32], bits)
+        k_hat, v_hat = O.dequant_record(rec, D, bits)
+        np.testing.assert_array_equal(per_c[g0:g0 + 32], k_hat)
+        np.testing.assert_array_equal(per_t[g0:g0 + 32], v_hat)
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_fake_quant_keys_exact_on_its_own_grid(bits):
+    rng = np.random.default_rng(50 + bits)
+    kc = _grid_tile(rng, 64, 64, bits, "k")
+    kt = _grid_tile(rng, 64, 64, bits, "v")
+    assert np.array_equal(O.fake_quant_keys(_bits(kc), bits, False), kc.numpy())
+    assert np.array_equal(O.fake_quant_keys(_bits(kt), bits, True), kt.numpy())
+    # and the other granularity is not exact on them
+    assert not np.array_equal(O.fake_quant_keys(_bits(kc), bits, True), kc.numpy())

@@ -50,6 +50,11 @@ def parse():
                    help="override the workload's layer count (small profiling captures)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--sweep", choices=["memory-wall"], default=None,
+                   help="memory-wall: decode attention of the 2-bit cache and of a bf16 cache "
+                        "over growing batches of the Llama-2-13B MHA 4K shape, until a cache "
+                        "no longer fits (one JSON line)")
+    p.add_argument("--sweep-batches", default="16,32,48,53,64,96,128,160,192,224,240,256")
     return p.parse_args()
 
 
@@ -601,8 +606,132 @@ def run_reference(args, w: synth.Workload, cfg: dict):
 
 # ---------------------------------------------------------------------------
 
+# ---------------------------------------------------------------------------
+# Memory-wall sweep: the 2-bit cache against a bf16 cache as the batch grows
+# ---------------------------------------------------------------------------
+
+def bf16_attention_bytes(B, H, Hq, D, S) -> int:
+    """bf16 K and V of S tokens + q in (bf16) + out (fp32), one layer."""
+    return B * H * S * D * 4 + B * Hq * D * (2 + 4)
+
+
+def _time_layers(call, layers, warmup=3, steps=10):
+    """Per-step device time (ms) of `call(layer)` over all layers; median of steps."""
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        for l in range(layers):
+            call(l)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for a, b in ev:
+        a.record(stream)
+        for l in range(layers):
+            call(l)
+        b.record(stream)
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) for a, b in ev)
+
+
+def _sweep_kivi(K, w, B, S, device, peak):
+    cfg = K.make_config(batch=B, num_layers=w.num_layers, num_kv_heads=w.num_kv_heads,
+                        num_q_heads=w.num_q_heads, head_dim=w.head_dim, bits=w.bits,
+                        max_tokens=S)
+    need = sum(getattr(K.kivi_required_bytes(cfg), f) for f in
+               ("records_bytes", "resid_k_bytes", "resid_v_bytes", "workspace_bytes"))
+    free = torch.cuda.mem_get_info()[0]
+    entry = {"impl": "kivi-2bit", "batch": B, "cache_gb": need / 1e9}
+    if need > free - (2 << 30):
+        return dict(entry, fits=False, free_gb=free / 1e9)
+    cache = K.KiviCache(batch=B, num_layers=w.num_layers, num_kv_heads=w.num_kv_heads,
+                        num_q_heads=w.num_q_heads, head_dim=w.head_dim, bits=w.bits,
+                        max_tokens=S, device=device)
+    # fill: a short prefill, then appends (no full-context staging buffer, so the
+    # cache alone has to fit); tokens cycle through a small seeded pool
+    wb = w.with_batch(B)
+    S0 = 160
+    pool = [synth.step_kv(wb, 0, i, device=device) for i in range(8)]
+    for l in range(w.num_layers):
+        k, v = synth.prefill_kv(wb, l, S=S0, device=device)
+        cache.prefill(l, k, v)
+        for t in range(S0, S):
+            kn, vn = pool[t % len(pool)]
+            cache.append(l, kn, vn)
+    q = [synth.query(wb, l, 0, device=device) for l in range(w.num_layers)]
+    out = torch.empty((B, w.num_q_heads, w.head_dim), dtype=torch.float32, device=device)
+    ms = _time_layers(lambda l: cache.attend(l, q[l], out), w.num_layers)
+    assert cache.check_device_status() == 0
+    cache.close()
+    del cache
+    nbytes = w.num_layers * attention_bytes(wb, S)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return dict(entry, fits=True, ms_per_step=ms, tokens_per_s=B / (ms * 1e-3),
+                gbs=gbs, frac_of_peak=gbs / peak)
+
+
+def _sweep_bf16(K, w, B, S, device, peak):
+    H, Hq, D, L = w.num_kv_heads, w.num_q_heads, w.head_dim, w.num_layers
+    Smax = S
+    need = 2 * L * B * H * Smax * D * 2
+    free = torch.cuda.mem_get_info()[0]
+    entry = {"impl": "bf16", "batch": B, "cache_gb": need / 1e9}
+    if need > free - (2 << 30):
+        return dict(entry, fits=False, free_gb=free / 1e9)
+    kc = torch.empty((L, B, H, Smax, D), dtype=torch.bfloat16, device=device)
+    vc = torch.empty_like(kc)
+    gen = torch.Generator(device=device).manual_seed(synth.BASE_SEED + 100 + B)
+    for l in range(L):
+        kc[l].normal_(generator=gen)
+        vc[l].normal_(generator=gen)
+    wb = w.with_batch(B)
+    q = [synth.query(wb, l, 0, device=device) for l in range(L)]
+    att = K.Bf16Attention(batch=B, num_kv_heads=H, num_q_heads=Hq, head_dim=D, device=device)
+    out = torch.empty((B, Hq, D), dtype=torch.float32, device=device)
+    ms = _time_layers(lambda l: att.attend(kc[l], vc[l], S, q[l], out), L)
+    assert att.check_device_status() == 0
+    del kc, vc
+    torch.cuda.empty_cache()
+    gbs = L * bf16_attention_bytes(B, H, Hq, D, S) / (ms * 1e-3) / 1e9
+    return dict(entry, fits=True, ms_per_step=ms, tokens_per_s=B / (ms * 1e-3),
+                gbs=gbs, frac_of_peak=gbs / peak)
+
+
+def run_memory_wall(args):
+    import decode_attention_kivi_b200 as K
+
+    device = torch.device("cuda", torch.cuda.current_device())
+    w = synth.WORKLOADS["llama2_13b_mha_sweep"]
+    S = w.context + 1
+    peak, peak_kind = hbm_peak()
+    rows = []
+    for impl, fn in (("bf16", _sweep_bf16), ("kivi-2bit", _sweep_kivi)):
+        for B in [int(x) for x in args.sweep_batches.split(",")]:
+            r = fn(K, w, B, S, device, peak)
+            rows.append(r)
+            torch.cuda.empty_cache()
+            print(json.dumps(r), file=sys.stderr, flush=True)
+            if not r["fits"]:
+                break
+    max_b = {i: max([r["batch"] for r in rows if r["impl"] == i and r["fits"]], default=0)
+             for i in ("bf16", "kivi-2bit")}
+    print(json.dumps({
+        "sweep": "memory-wall", "workload": w.name,
+        "shape": {"layers": w.num_layers, "heads": w.num_kv_heads, "head_dim": w.head_dim,
+                  "context_at_timed_call": S, "bits": w.bits},
+        "metric": "decode-attention tokens/s (all layers, attention calls only) and cache "
+                  "bytes that fit on one B200",
+        "peak_gbs": peak, "peak_kind": peak_kind, "rows": rows,
+        "largest_batch_that_fits": max_b,
+        "batch_ratio": max_b["kivi-2bit"] / max_b["bf16"] if max_b["bf16"] else None,
+        "data": "synthetic (seeded)",
+        "l2": "inputs larger than L2: one step reads every layer's cache"}), flush=True)
+
+
 def main():
     args = parse()
+    if args.sweep == "memory-wall":
+        run_memory_wall(args)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     w = synth.WORKLOADS[args.workload]

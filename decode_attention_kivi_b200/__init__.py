@@ -22,6 +22,8 @@ __all__ = [
     "kivi_cache_reset", "kivi_quantize_prefill", "kivi_append_token", "kivi_decode_attention",
     "kivi_check_device_status", "kivi_cache_bytes", "kivi_status_string",
     "kivi_decode_attention_static_scratch", "kivi_static_scratch_status",
+    "kivi_bf16_workspace_bytes", "kivi_bf16_decode_attention", "kivi_bf16_status",
+    "Bf16Attention", "kivi_fake_quant_keys",
 ]
 
 GROUP_SIZE = 32
@@ -151,6 +153,71 @@ def kivi_cache_bytes(cfg: KiviConfig, S: int) -> dict:
     check(lib().kivi_cache_bytes(ctypes.byref(cfg), S, ctypes.byref(a), ctypes.byref(b),
                                  ctypes.byref(c)), "kivi_cache_bytes")
     return {"stored": a.value, "codes_only": b.value, "convention": c.value}
+
+
+def kivi_bf16_workspace_bytes(batch: int, num_kv_heads: int, num_q_heads: int,
+                              head_dim: int) -> int:
+    n = ctypes.c_size_t()
+    check(lib().kivi_bf16_workspace_bytes(batch, num_kv_heads, num_q_heads, head_dim,
+                                          ctypes.byref(n)), "kivi_bf16_workspace_bytes")
+    return n.value
+
+
+def kivi_bf16_decode_attention(k_cache: torch.Tensor, v_cache: torch.Tensor, S: int,
+                               q: torch.Tensor, out: torch.Tensor, workspace: torch.Tensor,
+                               sm_scale: float = 0.0, stream=None) -> torch.Tensor:
+    """k_cache, v_cache: bf16 [B][Hkv][Smax][D]; q: bf16 [B][Hq][D]; out: fp32 like q."""
+    B, Hkv, Smax, D = k_cache.shape
+    Hq = q.shape[1]
+    if v_cache.shape != k_cache.shape or q.shape != (B, Hq, D) or out.shape != q.shape:
+        raise ValueError("shapes: k/v [B][Hkv][Smax][D], q and out [B][Hq][D]")
+    check(lib().kivi_bf16_decode_attention(
+        _ptr(k_cache, torch.bfloat16, "k_cache"), _ptr(v_cache, torch.bfloat16, "v_cache"),
+        B, Hkv, Hq, D, Smax, S, _ptr(q, torch.bfloat16, "q"), _ptr(out, torch.float32, "out"),
+        float(sm_scale), _ptr(workspace, name="workspace"),
+        workspace.numel() * workspace.element_size(), _stream(stream)),
+        "kivi_bf16_decode_attention")
+    return out
+
+
+def kivi_bf16_status(workspace: torch.Tensor, batch: int, num_kv_heads: int, stream=None) -> int:
+    code = ctypes.c_uint32()
+    rc = lib().kivi_bf16_status(_ptr(workspace, name="workspace"), batch, num_kv_heads,
+                                _stream(stream), ctypes.byref(code))
+    if rc not in (0, 7):
+        check(rc, "kivi_bf16_status")
+    return code.value
+
+
+def kivi_fake_quant_keys(k: torch.Tensor, bits: int, per_token: bool,
+                         k_hat: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Quantize-dequantize keys (bf16 [rows][D], rows a multiple of 32) per channel
+    (KIVI) or per token; returns fp32 k_hat [rows][D]."""
+    rows, D = k.shape
+    if k_hat is None:
+        k_hat = torch.empty((rows, D), dtype=torch.float32, device=k.device)
+    check(lib().kivi_fake_quant_keys(_ptr(k, torch.bfloat16, "k"), rows, D, bits,
+                                     int(bool(per_token)), _ptr(k_hat, torch.float32, "k_hat"),
+                                     _stream(stream)), "kivi_fake_quant_keys")
+    return k_hat
+
+
+class Bf16Attention:
+    """Owns the zeroed workspace of kivi_bf16_decode_attention for one shape."""
+
+    def __init__(self, *, batch, num_kv_heads, num_q_heads, head_dim, device=None):
+        self.B, self.Hkv, self.Hq, self.D = batch, num_kv_heads, num_q_heads, head_dim
+        n = kivi_bf16_workspace_bytes(batch, num_kv_heads, num_q_heads, head_dim)
+        self.workspace = torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+    def attend(self, k_cache, v_cache, S, q, out=None, sm_scale=0.0, stream=None):
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        return kivi_bf16_decode_attention(k_cache, v_cache, S, q, out, self.workspace, sm_scale,
+                                          stream)
+
+    def check_device_status(self, stream=None) -> int:
+        return kivi_bf16_status(self.workspace, self.B, self.Hkv, stream)
 
 
 def kivi_status_string(code: int) -> str:

@@ -66,6 +66,11 @@ def lib() -> ctypes.CDLL:
         "kivi_decode_attention_static_scratch": (st, [ctypes.POINTER(KiviConfig), P, P, P, I32,
                                                       I32, P, P, F32, P]),
         "kivi_static_scratch_status": (st, [P, ctypes.POINTER(ctypes.c_uint32)]),
+        "kivi_bf16_workspace_bytes": (st, [I32, I32, I32, I32, ctypes.POINTER(ctypes.c_size_t)]),
+        "kivi_bf16_decode_attention": (st, [P, P, I32, I32, I32, I32, I32, I32, P, P, F32, P,
+                                            ctypes.c_size_t, P]),
+        "kivi_bf16_status": (st, [P, I32, I32, P, ctypes.POINTER(ctypes.c_uint32)]),
+        "kivi_fake_quant_keys": (st, [P, ctypes.c_int64, I32, I32, I32, P, P]),
     }
     if hasattr(L, "kivi_debug_overstate_copies"):  # debug build only
         sig["kivi_debug_overstate_copies"] = (st, [ctypes.c_uint32])

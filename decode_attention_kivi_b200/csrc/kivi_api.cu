@@ -279,6 +279,103 @@ kivi_status kivi_check_device_status(kivi_cache* cache, void* stream, uint32_t* 
   return code ? KIVI_ERR_DEVICE : KIVI_OK;
 }
 
+// ---- the 16-bit baseline ----
+
+namespace {
+kivi_status bf16_shape(int32_t batch, int32_t hkv, int32_t hq, int32_t D) {
+  if (batch < 1 || hkv < 1 || hq < 1) return KIVI_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return KIVI_ERR_UNSUPPORTED;
+  if (hq % hkv != 0) return KIVI_ERR_UNSUPPORTED;
+  const int hpk = hq / hkv;
+  if (hpk != 1 && hpk != 2 && hpk != 4 && hpk != 8) return KIVI_ERR_UNSUPPORTED;
+  return KIVI_OK;
+}
+size_t bf16_fixed_bytes(int32_t batch, int32_t hkv) {
+  return kivi::kWsHeader + kivi::ws_tickets_bytes((long)batch * hkv);
+}
+}  // namespace
+
+kivi_status kivi_bf16_workspace_bytes(int32_t batch, int32_t num_kv_heads, int32_t num_q_heads,
+                                      int32_t head_dim, size_t* bytes) {
+  if (!bytes) return KIVI_ERR_INVALID_ARG;
+  const kivi_status st = bf16_shape(batch, num_kv_heads, num_q_heads, head_dim);
+  if (st != KIVI_OK) return st;
+  *bytes = bf16_fixed_bytes(batch, num_kv_heads) +
+           kivi::bf16_partial_bytes(head_dim, num_q_heads / num_kv_heads);
+  return KIVI_OK;
+}
+
+kivi_status kivi_bf16_decode_attention(const void* k_cache, const void* v_cache, int32_t batch,
+                                       int32_t num_kv_heads, int32_t num_q_heads,
+                                       int32_t head_dim, int32_t max_tokens, int32_t S,
+                                       const void* q, float* out, float sm_scale,
+                                       void* workspace, size_t workspace_bytes, void* stream) {
+  size_t need = 0;
+  const kivi_status st =
+      kivi_bf16_workspace_bytes(batch, num_kv_heads, num_q_heads, head_dim, &need);
+  if (st != KIVI_OK) return st;
+  if (!k_cache || !v_cache || !q || !out || !workspace) return KIVI_ERR_INVALID_ARG;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(q) || !aligned16(out) ||
+      !aligned16(workspace))
+    return KIVI_ERR_INVALID_ARG;
+  if (S < 1 || S > max_tokens || workspace_bytes < need || !std::isfinite(sm_scale))
+    return KIVI_ERR_INVALID_ARG;
+  if ((long)batch * num_kv_heads * max_tokens >= (1L << 31)) return KIVI_ERR_INVALID_ARG;
+  int device = 0, sms = 0;
+  if (cudaGetDevice(&device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
+    return KIVI_ERR_CUDA;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  kivi::Bf16DecodeArgs a{};
+  a.k = static_cast<const __nv_bfloat16*>(k_cache);
+  a.v = static_cast<const __nv_bfloat16*>(v_cache);
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.out = out;
+  a.status = reinterpret_cast<uint32_t*>(ws);
+  a.tickets = reinterpret_cast<int*>(ws + kivi::kWsHeader);
+  a.partials = reinterpret_cast<float*>(ws + bf16_fixed_bytes(batch, num_kv_heads));
+  a.B = batch;
+  a.Hkv = num_kv_heads;
+  a.Hq = num_q_heads;
+  a.D = head_dim;
+  a.Smax = max_tokens;
+  a.S = S;
+  a.sm_scale = sm_scale;
+  a.num_sms = sms;
+  a.device = device;
+  return from_cuda(kivi::launch_bf16_decode(a, static_cast<cudaStream_t>(stream)));
+}
+
+kivi_status kivi_bf16_status(void* workspace, int32_t batch, int32_t num_kv_heads, void* stream,
+                             uint32_t* code_out) {
+  if (!workspace || batch < 1 || num_kv_heads < 1) return KIVI_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return KIVI_ERR_CUDA;
+  uint32_t code = 0;
+  if (cudaMemcpy(&code, workspace, sizeof code, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return KIVI_ERR_CUDA;
+  if (code != 0 &&
+      cudaMemset(workspace, 0, bf16_fixed_bytes(batch, num_kv_heads)) != cudaSuccess)
+    return KIVI_ERR_CUDA;
+  if (code_out) *code_out = code;
+  return code ? KIVI_ERR_DEVICE : KIVI_OK;
+}
+
+// ---- key-granularity ablation ----
+
+kivi_status kivi_fake_quant_keys(const void* k, int64_t rows, int32_t head_dim, int32_t bits,
+                                 int32_t per_token, float* k_hat, void* stream) {
+  if (bits != 2 && bits != 4) return KIVI_ERR_UNSUPPORTED;
+  if (head_dim != 64 && head_dim != 128) return KIVI_ERR_UNSUPPORTED;
+  if (rows < 0 || rows % kGroup != 0) return KIVI_ERR_INVALID_ARG;
+  if (rows == 0) return KIVI_OK;
+  if (!k || !k_hat || !aligned16(k) || !aligned16(k_hat)) return KIVI_ERR_INVALID_ARG;
+  return from_cuda(kivi::launch_fake_quant_keys(head_dim, bits,
+                                                static_cast<const __nv_bfloat16*>(k), rows,
+                                                k_hat, per_token ? 1 : 0,
+                                                static_cast<cudaStream_t>(stream)));
+}
+
 kivi_status kivi_cache_bytes(const kivi_config* cfg, int32_t S, double* stored,
                              double* codes_only, double* convention) {
   kivi_status st = validate_config(cfg);

@@ -52,17 +52,13 @@
 
 #include "kivi_kernels.h"
 #include "kivi_launch.cuh"
+#include "kivi_ptx.cuh"
 #include "kivi_layout.cuh"
 
 namespace kivi {
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
-#ifdef KIVI_DEBUG_WAIT_CYCLES
-constexpr long long kWaitBudgetCycles = KIVI_DEBUG_WAIT_CYCLES;  // debug build: short waits
-#else
-constexpr long long kWaitBudgetCycles = 4000000000LL;  // about 2 s at 1.9 GHz
-#endif
 constexpr uint32_t kStatusWaitTimeout = 1u;
 constexpr uint32_t kStatusBadSplit = 4u;
 constexpr uint32_t kStatusBounds = 8u;  // debug build: an index outside its buffer (access skipped)
@@ -85,131 +81,6 @@ constexpr int kSmemBudget = 227 * 1024;
 #ifndef KIVI_MAX_WARPS
 #define KIVI_MAX_WARPS 16
 #endif
-
-// ---------------------------------------------------------------------------
-// PTX wrappers
-// ---------------------------------------------------------------------------
-
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
-               : "memory");
-}
-
-__device__ __forceinline__ void fence_mbar_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
-               "r"(bytes)
-               : "memory");
-}
-
-// Bulk copy global -> this CTA's shared memory, completing on `bar`.
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
-                                          uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(smem_addr(dst)),
-      "l"(src), "r"(bytes), "r"(smem_addr(bar))
-      : "memory");
-}
-
-// One test of the phase; the warp is suspended in hardware (not spinning) for
-// up to kSuspendHintNs while the phase is incomplete.
-constexpr uint32_t kSuspendHintNs = 1000000u;
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(done)
-      : "r"(smem_addr(bar)), "r"(parity), "r"(kSuspendHintNs)
-      : "memory");
-  return done != 0;
-}
-
-// Waits for phase `parity` of `bar` for at most kWaitBudgetCycles.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitBudgetCycles) return false;
-  }
-  return true;
-}
-
-__device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                        uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                         uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-
-__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-
-__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-
-__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;
-  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
-
-// (a & b) | c and (a & b) ^ c as one three-input logic op each.
-__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
-__device__ __forceinline__ uint32_t and_xor(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;
-  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
-
-__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
-  const __half2 h = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
-
-__device__ __forceinline__ float fast_exp2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
 
 // ---------------------------------------------------------------------------
 // Codes -> exact fp16 operands
@@ -334,7 +205,7 @@ struct Cfg {
   static constexpr int kThreads = kNW * 32;
   static constexpr int kSlots =
       cmin_i(64, (kSmemBudget - kFixed - kNW * kWarpBytes) / kSlotBytes);
-  static_assert(kNW >= 4 && kSlots >= kMinSlots, "shared-memory plan");
+  static_assert(kNW >= 4 && kNW <= 32 && kSlots >= kMinSlots, "shared-memory plan");
   static_assert(8 * kItemSlots * kNW + 16 + 8 * kNW + 12 * kSlots <= kFixed, "fixed area");
   static constexpr int kOffSlots = kNW * kWarpBytes;
   static constexpr int kOffFixed = kOffSlots + kSlots * kSlotBytes;
@@ -417,6 +288,45 @@ __host__ __device__ inline int cta_of_item(const Split& s, int it) {
 // ---------------------------------------------------------------------------
 // The decode kernel
 // ---------------------------------------------------------------------------
+
+// Segments: the items of one pair inside a CTA's range [it_begin, it_end).  With
+// at most NW segments every segment gets its own group of warps, so a warp never
+// leaves its pair: one warp each, and each of the other NW - n_pairs warps in
+// turn to the segment with the largest cost per warp (lane k of the calling warp
+// holds segment k; a warp-wide max picks the winner).  With more segments, each
+// warp sweeps a run of them.  Writes s_warp_seg[ww] = lo | hi << 16 for warp ww.
+// Kept out of line: its registers stay out of the decode loop's allocation.
+template <int NW>
+__device__ __noinline__ void segment_table(const Split& sp, int it_begin, int it_end, int p_first,
+                                           int n_pairs, int* s_warp_seg, int lane) {
+  if (n_pairs <= NW) {
+    int cost = 0, wk = 0;
+    if (lane < n_pairs) {
+      const int lo = lane == 0 ? item_cost_start(sp, it_begin) : (p_first + lane) * sp.pc;
+      const int hi = lane == n_pairs - 1 ? item_cost_start(sp, it_end) : (p_first + lane + 1) * sp.pc;
+      cost = hi - lo;
+      wk = 1;
+    }
+    for (int e = n_pairs; e < NW; ++e) {
+      // cost per warp as the bits of a positive float (ordered like the values),
+      // the low five bits replaced by the lane so that the lowest lane wins ties
+      const unsigned key =
+          lane < n_pairs ? (__float_as_uint(__fdividef((float)cost, (float)wk)) & ~31u) | (31u - lane)
+                         : 0u;
+      if (key == __reduce_max_sync(0xffffffffu, key) && lane < n_pairs) ++wk;
+    }
+    int first = wk;  // exclusive prefix of wk: the segment's first warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, first, o);
+      if (lane >= o) first += y;
+    }
+    first -= wk;
+    for (int j = 0; j < wk; ++j) s_warp_seg[first + j] = lane | ((lane + 1) << 16);
+  } else if (lane < NW) {
+    s_warp_seg[lane] = (lane * n_pairs / NW) | (((lane + 1) * n_pairs / NW) << 16);
+  }
+}
 
 template <int D, int BITS, int HPK>
 struct Warp;  // per-warp state and item processing (below)
@@ -883,34 +793,8 @@ decode_kernel(DecodeArgs args, Split sp) {
       s_seg_end[k] = min(it_end, (p_first + k + 1) * sp.ipp);
     }
   }
-  // Segments: the items of one pair inside this CTA's range.  With at most kNW
-  // segments every segment gets its own group of warps, sized by its cost, so a
-  // warp never leaves its pair; with more, each warp sweeps a run of segments.
-  // Thread 0 writes each warp's segment range [lo, hi) to s_warp_seg.
-  int* s_warp_seg = s_seg_end + C::kSlots;  // [kNW]: lo | hi << 16
-  if (threadIdx.x == 0) {
-    if (n_pairs <= C::kNW) {
-      int cost[C::kNW], wk[C::kNW];
-      for (int k = 0; k < n_pairs; ++k) {
-        const int a = max(it_begin, (p_first + k) * sp.ipp);
-        const int b = min(it_end, (p_first + k + 1) * sp.ipp);
-        cost[k] = item_cost_start(sp, b) - item_cost_start(sp, a);
-        wk[k] = 1;
-      }
-      for (int extra = C::kNW - n_pairs; extra > 0; --extra) {  // largest cost per warp first
-        int best = 0;
-        for (int k = 1; k < n_pairs; ++k)
-          if ((long)cost[k] * wk[best] > (long)cost[best] * wk[k]) best = k;
-        ++wk[best];
-      }
-      int ww = 0;
-      for (int k = 0; k < n_pairs; ++k)
-        for (int j = 0; j < wk[k]; ++j, ++ww) s_warp_seg[ww] = k | ((k + 1) << 16);
-    } else {
-      for (int ww = 0; ww < C::kNW; ++ww)
-        s_warp_seg[ww] = (ww * n_pairs / C::kNW) | (((ww + 1) * n_pairs / C::kNW) << 16);
-    }
-  }
+  int* s_warp_seg = s_seg_end + C::kSlots;  // [kNW]: warp ww's segments lo | hi << 16
+  if (warp == 0) segment_table<C::kNW>(sp, it_begin, it_end, p_first, n_pairs, s_warp_seg, lane);
   int seg_cur = 0, seg_hi = 0;  // this warp's segments, read after the barrier below
   const int NG = sp.NG, S = args.S;
   const long rec_stride = C::kRec;

@@ -60,6 +60,29 @@ long decode_workspace_bytes(int D, int bits, int hpk, long pairs);
 // of the decode kernel; cudaErrorNotSupported in a regular build.
 cudaError_t debug_overstate_copies(unsigned bytes);
 
+// Decode attention over an unquantized bf16 cache [B][Hkv][Smax][D] (tokens
+// 0..S-1): the 16-bit baseline.  Workspace: status header, tickets, then
+// bf16_partial_bytes of split partials.
+struct Bf16DecodeArgs {
+  const __nv_bfloat16 *k, *v;  // one layer's cache
+  const __nv_bfloat16* q;      // [B][Hq][D]
+  float* out;                  // [B][Hq][D]
+  uint32_t* status;            // workspace header
+  int* tickets;                // [B * Hkv], zero between calls
+  float* partials;
+  int B, Hkv, Hq, D, Smax, S;
+  float sm_scale;              // <= 0: 1/sqrt(D)
+  int num_sms;
+  int device;
+};
+long bf16_partial_bytes(int D, int hpk);
+cudaError_t launch_bf16_decode(const Bf16DecodeArgs& a, cudaStream_t stream);
+
+// Key-granularity ablation: quantize-dequantize keys [rows][D] (rows a multiple
+// of 32) per channel or per token into fp32 k_hat.
+cudaError_t launch_fake_quant_keys(int D, int bits, const __nv_bfloat16* k, long rows,
+                                   float* k_hat, int per_token, cudaStream_t stream);
+
 cudaError_t launch_prefill(int D, int bits, const PrefillArgs& a, cudaStream_t stream);
 cudaError_t launch_append(int D, int bits, const AppendArgs& a, cudaStream_t stream);
 cudaError_t launch_decode(int D, int bits, const DecodeArgs& a, cudaStream_t stream);

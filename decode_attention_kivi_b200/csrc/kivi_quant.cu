@@ -54,11 +54,27 @@ __device__ __forceinline__ void load_tile(__nv_bfloat16 (*dst)[D], const __nv_bf
   }
 }
 
+// (min, scale) of the n values x[0], x[stride], ...: exact min and max, then
+// scale = (max - min) / (2^b - 1) rounded to nearest.
+template <int BITS>
+__device__ __forceinline__ void group_params(const __nv_bfloat16* x, int n, int stride, float& mn,
+                                             float& scale) {
+  constexpr int kQmax = (1 << BITS) - 1;
+  mn = __bfloat162float(x[0]);
+  float mx = mn;
+#pragma unroll 8
+  for (int i = 1; i < n; ++i) {
+    const float v = __bfloat162float(x[i * stride]);
+    mn = v < mn ? v : mn;  // strict comparisons, first occurrence wins (signed zeros)
+    mx = v > mx ? v : mx;
+  }
+  scale = __fdiv_rn(__fsub_rn(mx, mn), (float)kQmax);
+}
+
 // Quantizes the K and V tiles in smem into one group record at `rec`.
 template <int D, int BITS>
 __device__ void quantize_tiles_to_record(QuantSmem<D>& sm, uint32_t* __restrict__ rec) {
   constexpr RecordGeom geo{D, BITS};
-  constexpr int kQmax = (1 << BITS) - 1;
   unsigned short* rec16 = reinterpret_cast<unsigned short*>(rec);
   unsigned short* kscale = rec16 + geo.k_scale_off() / 2;
   unsigned short* kmin = rec16 + geo.k_min_off() / 2;
@@ -66,14 +82,8 @@ __device__ void quantize_tiles_to_record(QuantSmem<D>& sm, uint32_t* __restrict_
   unsigned short* vmin = rec16 + geo.v_min_off() / 2;
   // Keys: per channel d over the 32 tokens.
   for (int d = threadIdx.x; d < D; d += kQuantThreads) {
-    float mn = __bfloat162float(sm.k[0][d]), mx = mn;
-#pragma unroll 8
-    for (int t = 1; t < kGroup; ++t) {
-      const float x = __bfloat162float(sm.k[t][d]);
-      mn = x < mn ? x : mn;  // strict comparisons, first occurrence wins (signed zeros)
-      mx = x > mx ? x : mx;
-    }
-    const float scale = __fdiv_rn(__fsub_rn(mx, mn), (float)kQmax);
+    float mn, scale;
+    group_params<BITS>(&sm.k[0][d], kGroup, D, mn, scale);
 #pragma unroll 8
     for (int t = 0; t < kGroup; ++t) sm.kc[t][d] = quant_code<BITS>(__bfloat162float(sm.k[t][d]), mn, scale);
     kscale[d] = to_f16_bits(scale);
@@ -83,14 +93,8 @@ __device__ void quantize_tiles_to_record(QuantSmem<D>& sm, uint32_t* __restrict_
   constexpr int kBlocks = D / 32;
   for (int p = threadIdx.x; p < kGroup * kBlocks; p += kQuantThreads) {
     const int t = p / kBlocks, j = p % kBlocks;
-    float mn = __bfloat162float(sm.v[t][32 * j]), mx = mn;
-#pragma unroll 8
-    for (int c = 1; c < 32; ++c) {
-      const float x = __bfloat162float(sm.v[t][32 * j + c]);
-      mn = x < mn ? x : mn;
-      mx = x > mx ? x : mx;
-    }
-    const float scale = __fdiv_rn(__fsub_rn(mx, mn), (float)kQmax);
+    float mn, scale;
+    group_params<BITS>(&sm.v[t][32 * j], 32, 1, mn, scale);
 #pragma unroll 8
     for (int c = 0; c < 32; ++c)
       sm.vc[t][32 * j + c] = quant_code<BITS>(__bfloat162float(sm.v[t][32 * j + c]), mn, scale);
@@ -212,6 +216,45 @@ append_kernel(const __nv_bfloat16* __restrict__ k_new, const __nv_bfloat16* __re
   }
 }
 
+// Key-granularity ablation: quantize-dequantize the keys of one 32-token group,
+// per channel (KIVI's rule for keys) or per token over 32-channel blocks (the
+// values' rule), with the record's quantizer and fp16 metadata;
+// k_hat = RN(fp16(scale) * code + fp16(min)) in fp32 (one rounding).
+template <int D, int BITS>
+__global__ void __launch_bounds__(kQuantThreads)
+fake_quant_keys_kernel(const __nv_bfloat16* __restrict__ k, float* __restrict__ k_hat,
+                       int per_token) {
+  __shared__ __align__(16) __nv_bfloat16 tile[kGroup][D];
+  const long row0 = (long)blockIdx.x * kGroup;
+  wait_for_predecessor();
+  load_tile<D>(tile, k + row0 * D, D);
+  __syncthreads();
+  allow_successor();
+  const int n_groups = per_token ? kGroup * (D / 32) : D;
+  for (int u = threadIdx.x; u < n_groups; u += kQuantThreads) {
+    // group u: channel u of the 32 tokens, or token u / (D/32), channels 32 (u % (D/32)) + i
+    const int t0 = per_token ? u / (D / 32) : 0, d0 = per_token ? 32 * (u % (D / 32)) : u;
+    const int stride = per_token ? 1 : D;
+    const __nv_bfloat16* x = &tile[t0][d0];
+    float mn, scale;
+    group_params<BITS>(x, 32, stride, mn, scale);
+    const float sh = __half2float(__float2half_rn(scale)), mh = __half2float(__float2half_rn(mn));
+    for (int i = 0; i < 32; ++i) {
+      const int c = quant_code<BITS>(__bfloat162float(x[i * stride]), mn, scale);
+      k_hat[(row0 + t0) * D + d0 + (long)i * stride] = __fmaf_rn(sh, (float)c, mh);
+    }
+  }
+}
+
+template <int D, int BITS>
+cudaError_t launch_fake_quant_t(const __nv_bfloat16* k, long rows, float* k_hat, int per_token,
+                                cudaStream_t stream) {
+  if (rows % kGroup != 0 || rows / kGroup > 0x7fffffffL) return cudaErrorInvalidValue;
+  cudaError_t e = launch_pdl(fake_quant_keys_kernel<D, BITS>, dim3((unsigned)(rows / kGroup)),
+                             dim3(kQuantThreads), 0, stream, k, k_hat, per_token);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 template <int D, int BITS>
 cudaError_t launch_prefill_t(const PrefillArgs& a, cudaStream_t stream) {
   if (a.ng > 0) {
@@ -238,6 +281,16 @@ cudaError_t launch_append_t(const AppendArgs& a, cudaStream_t stream) {
 }
 
 }  // namespace
+
+cudaError_t launch_fake_quant_keys(int D, int bits, const __nv_bfloat16* k, long rows,
+                                   float* k_hat, int per_token, cudaStream_t stream) {
+  if (rows == 0) return cudaSuccess;
+  if (D == 128 && bits == 2) return launch_fake_quant_t<128, 2>(k, rows, k_hat, per_token, stream);
+  if (D == 128 && bits == 4) return launch_fake_quant_t<128, 4>(k, rows, k_hat, per_token, stream);
+  if (D == 64 && bits == 2) return launch_fake_quant_t<64, 2>(k, rows, k_hat, per_token, stream);
+  if (D == 64 && bits == 4) return launch_fake_quant_t<64, 4>(k, rows, k_hat, per_token, stream);
+  return cudaErrorInvalidValue;
+}
 
 cudaError_t launch_prefill(int D, int bits, const PrefillArgs& a, cudaStream_t stream) {
   if (D == 128 && bits == 2) return launch_prefill_t<128, 2>(a, stream);

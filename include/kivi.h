@@ -240,6 +240,75 @@ kivi_status kivi_check_device_status(kivi_cache* cache, void* stream,
 kivi_status kivi_cache_bytes(const kivi_config* cfg, int32_t S, double* stored,
                              double* codes_only, double* convention);
 
+/* ------------------------------------------------------------------------ */
+/* The 16-bit baseline: decode attention over an unquantized bf16 cache      */
+/* ------------------------------------------------------------------------ */
+
+/* Workspace bytes of kivi_bf16_decode_attention for `batch` sequences of
+ * `num_kv_heads` kv heads and `num_q_heads` query heads of `head_dim`: a status
+ * header (256 B), one ticket per (sequence, kv head) rounded up to 256 B, and
+ * the split partials of up to 256 CTAs.  Host only.  The buffer must be
+ * zero-filled before its first use; every call leaves it zeroed again except
+ * for the status word after a failure (cleared by kivi_bf16_status).
+ * Errors: INVALID_ARG, UNSUPPORTED (head_dim not 64/128, num_q_heads /
+ * num_kv_heads not 1, 2, 4 or 8). */
+kivi_status kivi_bf16_workspace_bytes(int32_t batch, int32_t num_kv_heads,
+                                      int32_t num_q_heads, int32_t head_dim,
+                                      size_t* bytes);
+
+/* Decode attention over an unquantized bf16 KV cache: the full-precision
+ * baseline the [KIVI page] and the [HF page] compare the 2-bit cache with.
+ * For query head h of sequence b (kv head h / (num_q_heads / num_kv_heads)),
+ *   out[b][h] = sum_{t<S} softmax_t(sm_scale * <q[b][h], k[b][kvh][t]>) v[b][kvh][t].
+ *   k_cache, v_cache: bf16 [batch][num_kv_heads][max_tokens][head_dim] (one
+ *       layer), device, 16-byte aligned, owned by the caller; tokens S and
+ *       beyond are never read into the result (they may hold anything).
+ *   q: bf16 [batch][num_q_heads][head_dim]; out: fp32, same shape.
+ *   sm_scale <= 0 means 1/sqrt(head_dim).
+ *   workspace: kivi_bf16_workspace_bytes bytes (see there).
+ * Asynchronous on `stream`; allocates nothing.  Calls that share a workspace
+ * must not overlap on the GPU.
+ * Errors: INVALID_ARG (NULL or unaligned pointers, S < 1 or S > max_tokens,
+ * batch * num_kv_heads * max_tokens >= 2^31, workspace too small, sm_scale not
+ * finite), UNSUPPORTED, CUDA. */
+kivi_status kivi_bf16_decode_attention(const void* k_cache, const void* v_cache,
+                                       int32_t batch, int32_t num_kv_heads,
+                                       int32_t num_q_heads, int32_t head_dim,
+                                       int32_t max_tokens, int32_t S, const void* q,
+                                       float* out, float sm_scale, void* workspace,
+                                       size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, reads the status word of a kivi_bf16_decode_attention
+ * workspace and, if it is not zero, clears the header and the tickets of
+ * `batch` x `num_kv_heads` pairs.  KIVI_ERR_DEVICE if a bounded wait ran out,
+ * KIVI_ERR_CUDA if a CUDA call failed, else KIVI_OK; `code_out` may be NULL. */
+kivi_status kivi_bf16_status(void* workspace, int32_t batch, int32_t num_kv_heads,
+                             void* stream, uint32_t* code_out);
+
+/* ------------------------------------------------------------------------ */
+/* Key-granularity ablation                                                  */
+/* ------------------------------------------------------------------------ */
+
+/* Quantizes and dequantizes keys with `bits` bits at one of two granularities,
+ * to measure the claim of the [KIVI page] and the [HF page] that keys, whose
+ * magnitudes concentrate in a few outlier channels, must be quantized per
+ * channel and not per token:
+ *   per_token == 0: KIVI's key rule, one group per channel of every 32
+ *       consecutive rows (tokens), as in the group record;
+ *   per_token != 0: one group per row over each block of 32 channels (the
+ *       values' rule applied to keys).
+ * The quantizer is the record's (min/max zero point, fp32 scale, codes round
+ * half to even, fp16 metadata); k_hat = fp16(scale) * code + fp16(min) rounded
+ * once to fp32.
+ *   k: bf16 [rows][head_dim], device, 16-byte aligned; rows a multiple of 32
+ *      (rows of several sequences may be stacked: groups never straddle 32).
+ *   k_hat: fp32 [rows][head_dim], device, written.
+ * Asynchronous on `stream`.  Errors: INVALID_ARG (NULL or unaligned pointers,
+ * rows < 0 or not a multiple of 32), UNSUPPORTED (bits not 2/4, head_dim not
+ * 64/128), CUDA. */
+kivi_status kivi_fake_quant_keys(const void* k, int64_t rows, int32_t head_dim, int32_t bits,
+                                 int32_t per_token, float* k_hat, void* stream);
+
 /* Static text for a status code; never NULL. */
 const char* kivi_status_string(kivi_status status);
 

@@ -133,3 +133,35 @@ def test_cache_bytes_pages_numbers(lib):
     lib.kivi_cache_bytes(ctypes.byref(c), 8192, None, None, ctypes.byref(out[2]))
     assert out[2].value == 34816
     assert lib.kivi_cache_bytes(ctypes.byref(c), 0, None, None, None) == 1
+
+
+def test_bf16_workspace_bytes_and_validation(lib):
+    """The bf16 baseline's host checks (no launch happens on these paths)."""
+    n = ctypes.c_size_t()
+    assert lib.kivi_bf16_workspace_bytes(16, 8, 32, 128, ctypes.byref(n)) == 0
+    # header, 128 tickets rounded to 256 bytes, 256 CTAs x 2 partials of 4 heads
+    assert n.value == 256 + 512 + 256 * 2 * 4 * 130 * 4
+    assert N.STATUS[lib.kivi_bf16_workspace_bytes(1, 8, 24, 128, ctypes.byref(n))] == \
+        "KIVI_ERR_UNSUPPORTED"
+    assert N.STATUS[lib.kivi_bf16_workspace_bytes(1, 8, 8, 96, ctypes.byref(n))] == \
+        "KIVI_ERR_UNSUPPORTED"
+    fake = 1 << 20
+    call = lambda S, Smax, ws: lib.kivi_bf16_decode_attention(  # noqa: E731
+        fake, fake, 2, 2, 4, 128, Smax, S, fake, fake, 0.0, fake, ws, None)
+    assert N.STATUS[call(0, 10, 1 << 30)] == "KIVI_ERR_INVALID_ARG"     # S < 1
+    assert N.STATUS[call(11, 10, 1 << 30)] == "KIVI_ERR_INVALID_ARG"    # S > max_tokens
+    assert N.STATUS[call(5, 10, 100)] == "KIVI_ERR_INVALID_ARG"         # workspace too small
+    assert N.STATUS[lib.kivi_bf16_decode_attention(
+        fake + 2, fake, 2, 2, 4, 128, 10, 5, fake, fake, 0.0, fake, 1 << 30, None)] == \
+        "KIVI_ERR_INVALID_ARG"                                             # unaligned
+
+
+def test_fake_quant_keys_validation(lib):
+    fake = 1 << 20
+    assert N.STATUS[lib.kivi_fake_quant_keys(fake, 33, 128, 2, 0, fake, None)] == \
+        "KIVI_ERR_INVALID_ARG"
+    assert N.STATUS[lib.kivi_fake_quant_keys(fake, 32, 128, 3, 0, fake, None)] == \
+        "KIVI_ERR_UNSUPPORTED"
+    assert N.STATUS[lib.kivi_fake_quant_keys(fake, 32, 96, 2, 0, fake, None)] == \
+        "KIVI_ERR_UNSUPPORTED"
+    assert lib.kivi_fake_quant_keys(fake, 0, 128, 2, 1, fake, None) == 0  # nothing to do

@@ -11,14 +11,18 @@
 // Work: one persistent CTA per SM.  The work of a (sequence, kv head) pair is a
 // list of items: pairs of group records (64 tokens), a last single record, and
 // residual items of 8 ring tokens.  The items of all pairs, in order, are split
-// into one contiguous range per CTA, balanced by their bytes; inside a CTA the
-// warps claim items from a shared counter, so warps that run ahead take more.
-// Each warp streams its items into its own two-item shared-memory ring with
-// cp.async.bulk on mbarriers and keeps one online-softmax state per pair; when
-// it moves to another pair it merges that state into the CTA's slot for the
-// pair.  At the end each CTA writes the output of the pairs it holds whole; for
-// a pair shared with other CTAs it writes a partial, and the last CTA to
-// arrive (a ticket per pair) merges the partials into the output.
+// into one contiguous range per CTA, balanced by their bytes.  Inside a CTA the
+// items of one pair form a segment; each segment gets its own group of warps
+// (sized by the segment's cost), and the warps of a group claim its items from
+// the segment's counter, so warps that run ahead take more.  Each warp streams
+// its items into its own two-item shared-memory ring with cp.async.bulk on
+// mbarriers and keeps one online-softmax state.  A warp that has to move to
+// another pair (only when a CTA holds more segments than warps) parks its state
+// in its own global slot, without a lock.  At the end the warps' final and
+// parked states of each pair are merged; each CTA writes the output of the
+// pairs it holds whole, and for a pair shared with other CTAs it writes a
+// partial: the last CTA to arrive (a ticket per pair) merges the partials into
+// the output.
 //
 // Group records, on the tensor cores (mma.sync m16n8k16, fp16 operands, fp32
 // accumulation):
@@ -44,9 +48,9 @@
 // products): scores with q itself, P.V with p as a bf16 hi + lo pair in the two
 // halves of the k dimension.
 //
-// Every wait is bounded: a wait on an mbarrier or a lock that runs out sets the
-// device status word and the warp stops issuing work; the CTA still finishes
-// its bookkeeping so that no other CTA waits on it.
+// Every wait is bounded: a wait on an mbarrier that runs out sets the device
+// status word and the warp stops issuing work; the CTA still finishes its
+// bookkeeping so that no other CTA waits on it.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -288,45 +292,6 @@ __host__ __device__ inline int cta_of_item(const Split& s, int it) {
 // ---------------------------------------------------------------------------
 // The decode kernel
 // ---------------------------------------------------------------------------
-
-// Segments: the items of one pair inside a CTA's range [it_begin, it_end).  With
-// at most NW segments every segment gets its own group of warps, so a warp never
-// leaves its pair: one warp each, and each of the other NW - n_pairs warps in
-// turn to the segment with the largest cost per warp (lane k of the calling warp
-// holds segment k; a warp-wide max picks the winner).  With more segments, each
-// warp sweeps a run of them.  Writes s_warp_seg[ww] = lo | hi << 16 for warp ww.
-// Kept out of line: its registers stay out of the decode loop's allocation.
-template <int NW>
-__device__ __noinline__ void segment_table(const Split& sp, int it_begin, int it_end, int p_first,
-                                           int n_pairs, int* s_warp_seg, int lane) {
-  if (n_pairs <= NW) {
-    int cost = 0, wk = 0;
-    if (lane < n_pairs) {
-      const int lo = lane == 0 ? item_cost_start(sp, it_begin) : (p_first + lane) * sp.pc;
-      const int hi = lane == n_pairs - 1 ? item_cost_start(sp, it_end) : (p_first + lane + 1) * sp.pc;
-      cost = hi - lo;
-      wk = 1;
-    }
-    for (int e = n_pairs; e < NW; ++e) {
-      // cost per warp as the bits of a positive float (ordered like the values),
-      // the low five bits replaced by the lane so that the lowest lane wins ties
-      const unsigned key =
-          lane < n_pairs ? (__float_as_uint(__fdividef((float)cost, (float)wk)) & ~31u) | (31u - lane)
-                         : 0u;
-      if (key == __reduce_max_sync(0xffffffffu, key) && lane < n_pairs) ++wk;
-    }
-    int first = wk;  // exclusive prefix of wk: the segment's first warp
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, first, o);
-      if (lane >= o) first += y;
-    }
-    first -= wk;
-    for (int j = 0; j < wk; ++j) s_warp_seg[first + j] = lane | ((lane + 1) << 16);
-  } else if (lane < NW) {
-    s_warp_seg[lane] = (lane * n_pairs / NW) | (((lane + 1) * n_pairs / NW) << 16);
-  }
-}
 
 template <int D, int BITS, int HPK>
 struct Warp;  // per-warp state and item processing (below)
@@ -793,8 +758,34 @@ decode_kernel(DecodeArgs args, Split sp) {
       s_seg_end[k] = min(it_end, (p_first + k + 1) * sp.ipp);
     }
   }
-  int* s_warp_seg = s_seg_end + C::kSlots;  // [kNW]: warp ww's segments lo | hi << 16
-  if (warp == 0) segment_table<C::kNW>(sp, it_begin, it_end, p_first, n_pairs, s_warp_seg, lane);
+  // Segments: the items of one pair inside this CTA's range.  With at most kNW
+  // segments every segment gets its own group of warps, sized by its cost, so a
+  // warp never leaves its pair; with more, each warp sweeps a run of segments.
+  // Thread 0 writes each warp's segment range [lo, hi) to s_warp_seg.
+  int* s_warp_seg = s_seg_end + C::kSlots;  // [kNW]: lo | hi << 16
+  if (threadIdx.x == 0) {
+    if (n_pairs <= C::kNW) {
+      int cost[C::kNW], wk[C::kNW];
+      for (int k = 0; k < n_pairs; ++k) {
+        const int a = max(it_begin, (p_first + k) * sp.ipp);
+        const int b = min(it_end, (p_first + k + 1) * sp.ipp);
+        cost[k] = item_cost_start(sp, b) - item_cost_start(sp, a);
+        wk[k] = 1;
+      }
+      for (int extra = C::kNW - n_pairs; extra > 0; --extra) {  // largest cost per warp first
+        int best = 0;
+        for (int k = 1; k < n_pairs; ++k)
+          if ((long)cost[k] * wk[best] > (long)cost[best] * wk[k]) best = k;
+        ++wk[best];
+      }
+      int ww = 0;
+      for (int k = 0; k < n_pairs; ++k)
+        for (int j = 0; j < wk[k]; ++j, ++ww) s_warp_seg[ww] = k | ((k + 1) << 16);
+    } else {
+      for (int ww = 0; ww < C::kNW; ++ww)
+        s_warp_seg[ww] = (ww * n_pairs / C::kNW) | (((ww + 1) * n_pairs / C::kNW) << 16);
+    }
+  }
   int seg_cur = 0, seg_hi = 0;  // this warp's segments, read after the barrier below
   const int NG = sp.NG, S = args.S;
   const long rec_stride = C::kRec;

@@ -18,11 +18,13 @@
 // its items into its own two-item shared-memory ring with cp.async.bulk on
 // mbarriers and keeps one online-softmax state.  A warp that has to move to
 // another pair (only when a CTA holds more segments than warps) parks its state
-// in its own global slot, without a lock.  At the end the warps' final and
-// parked states of each pair are merged; each CTA writes the output of the
-// pairs it holds whole, and for a pair shared with other CTAs it writes a
-// partial: the last CTA to arrive (a ticket per pair) merges the partials into
-// the output.
+// in its own global slot, without a lock.  At the end the last warp of each
+// segment's group to finish merges the group's final states on its own (no
+// CTA-wide barrier, so it overlaps the other groups' items); with more segments
+// than warps, all threads merge the final and parked states after one barrier.
+// A pair held whole goes to the output; for a pair shared with other CTAs the
+// CTA writes a partial, and the last CTA to arrive (a ticket per pair) merges
+// the partials into the output.
 //
 // Group records, on the tensor cores (mma.sync m16n8k16, fp16 operands, fp32
 // accumulation):
@@ -210,7 +212,7 @@ struct Cfg {
   static constexpr int kSlots =
       cmin_i(64, (kSmemBudget - kFixed - kNW * kWarpBytes) / kSlotBytes);
   static_assert(kNW >= 4 && kNW <= 32 && kSlots >= kMinSlots, "shared-memory plan");
-  static_assert(8 * kItemSlots * kNW + 16 + 8 * kNW + 12 * kSlots <= kFixed, "fixed area");
+  static_assert(8 * kItemSlots * kNW + 16 + 8 * kNW + 20 * kSlots <= kFixed, "fixed area");
   static constexpr int kOffSlots = kNW * kWarpBytes;
   static constexpr int kOffFixed = kOffSlots + kSlots * kSlotBytes;
   static constexpr int kBytes = kOffFixed + kFixed;
@@ -649,6 +651,7 @@ struct Warp {
         *reinterpret_cast<uint4*>(base + C::kRec + t * C::kResRow + 16 * c) =
             make_uint4(0u, 0u, 0u, 0u);
       }
+      fence_proxy_async();  // the slot's next bulk copy comes after these writes
       __syncwarp();
     }
     // scores: rows = tokens (0..7), columns 2h = head 4c + h (q in bf16), 2h+1 = 0
@@ -738,6 +741,8 @@ decode_kernel(DecodeArgs args, Split sp) {
   unsigned* s_parked = reinterpret_cast<unsigned*>(s_final + C::kNW);  // [kSlots] warp bitmasks
   int* s_seg_next = reinterpret_cast<int*>(s_parked + C::kSlots);      // [kSlots] claim counters
   int* s_seg_end = s_seg_next + C::kSlots;                             // [kSlots] end items
+  int* s_gsize = s_seg_end + C::kSlots + C::kNW;  // [kSlots] warps of each segment (after s_warp_seg)
+  int* s_done = s_gsize + C::kSlots;              // [kSlots] warps of each segment that finished
   if (it_end <= it_begin || n_pairs > C::kSlots) {  // the host's split rules exclude both
     if (threadIdx.x == 0) atomicOr(args.status, kStatusBadSplit);
     return;
@@ -754,6 +759,7 @@ decode_kernel(DecodeArgs args, Split sp) {
     }
     for (int k = threadIdx.x; k < n_pairs; k += C::kThreads) {
       s_parked[k] = 0u;
+      s_done[k] = 0;
       s_seg_next[k] = max(it_begin, (p_first + k) * sp.ipp);
       s_seg_end[k] = min(it_end, (p_first + k + 1) * sp.ipp);
     }
@@ -779,8 +785,10 @@ decode_kernel(DecodeArgs args, Split sp) {
         ++wk[best];
       }
       int ww = 0;
-      for (int k = 0; k < n_pairs; ++k)
+      for (int k = 0; k < n_pairs; ++k) {
+        s_gsize[k] = wk[k];
         for (int j = 0; j < wk[k]; ++j, ++ww) s_warp_seg[ww] = k | ((k + 1) << 16);
+      }
     } else {
       for (int ww = 0; ww < C::kNW; ++ww)
         s_warp_seg[ww] = (ww * n_pairs / C::kNW) | (((ww + 1) * n_pairs / C::kNW) << 16);
@@ -874,6 +882,112 @@ decode_kernel(DecodeArgs args, Split sp) {
   }
   w.reset();
 
+  // The partial of CTA ct for `pair`: side 0 if the pair is ct's first pair.
+  auto partial_of = [&](int ct, int pair) -> float* {
+    return args.partials + ((long)ct * 2 + (pair == cta_first_item(sp, ct) / sp.ipp ? 0 : 1)) *
+                               (long)(HPK * (D + 2));
+  };
+  // Merges, with this warp alone, the final states of segment `seg`'s warps (all
+  // of them have counted themselves done) and writes the pair's output, or this
+  // CTA's partial and the pair's ticket; the CTA that takes the last ticket of a
+  // shared pair merges the pair's partials.
+  auto merge_segment = [&](int seg) {
+    constexpr int kEl = HPK * D / 32;  // elements of a state per lane: e = lane + 32 i
+    const int pair = p_first + seg;
+    float* tab = reinterpret_cast<float*>(wbase + C::kItemSlots * C::kItemBytes);  // own p tile
+    float* s_M = tab + C::kNW * HPK;  // [HPK] merged max, then [HPK] merged sum
+    // lane ww < kNW: warp ww's factors 2^(m - M) per head (0 when not in the group)
+    const int wl = min(lane, C::kNW - 1);
+    const bool member = lane < C::kNW && (s_warp_seg[wl] & 0xffff) == seg && s_final[wl] == seg;
+    const unsigned members = __ballot_sync(0xffffffffu, member);
+    const float* st = reinterpret_cast<const float*>(smem + wl * C::kWarpBytes);
+#pragma unroll
+    for (int h = 0; h < HPK; ++h) {
+      const float m = member ? st[h] : -INFINITY;
+      float M = m;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+      const float f = member ? exp2f(m - M) : 0.f;
+      float L = member ? f * st[HPK + h] : 0.f;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+      if (lane < C::kNW) tab[lane * HPK + h] = f;
+      if (lane == 0) {
+        s_M[h] = M;
+        s_M[HPK + h] = L;
+      }
+    }
+    __syncwarp();
+    // acc: the member warps one after another, all of a lane's elements at once
+    float A[kEl];
+#pragma unroll
+    for (int i = 0; i < kEl; ++i) A[i] = 0.f;
+    for (unsigned mm = members; mm; mm &= mm - 1) {
+      const int ww = __ffs(mm) - 1;
+      const float* src = reinterpret_cast<const float*>(smem + ww * C::kWarpBytes) + 2 * HPK;
+#pragma unroll
+      for (int i = 0; i < kEl; ++i) A[i] = fmaf(tab[ww * HPK + (lane + 32 * i) / D], src[lane + 32 * i], A[i]);
+    }
+    const int fc = cta_of_item(sp, pair * sp.ipp), lc = cta_of_item(sp, pair * sp.ipp + sp.ipp - 1);
+    const int b = pair / args.Hkv, kvh = pair % args.Hkv;
+    float* out = args.out + ((long)b * args.Hq + (long)kvh * HPK) * D;
+    if (fc == lc) {  // held whole by this CTA
+#pragma unroll
+      for (int i = 0; i < kEl; ++i) out[lane + 32 * i] = A[i] / s_M[HPK + (lane + 32 * i) / D];
+      return;
+    }
+    if (cta >= args.max_ctas) {  // the host's split rules exclude this
+      if (lane == 0) atomicOr(args.status, kStatusBadSplit);
+      return;
+    }
+    float* part = partial_of(cta, pair);
+#pragma unroll
+    for (int i = 0; i < kEl; ++i) part[2 * HPK + lane + 32 * i] = A[i];
+    if (lane < HPK) {
+      part[lane] = s_M[lane];
+      part[HPK + lane] = s_M[HPK + lane];
+    }
+    __threadfence();  // the partial before the ticket
+    __syncwarp();
+    int is_last = 0;
+    if (lane == 0) is_last = atomicAdd(&args.tickets[pair], 1) == lc - fc;
+    is_last = __shfl_sync(0xffffffffu, is_last, 0);
+    if (!is_last) return;
+    __threadfence();
+    // the pair's partials, CTA by CTA (online), all of a lane's elements at once
+    float Mh[HPK], Lh[HPK];
+#pragma unroll
+    for (int h = 0; h < HPK; ++h) {
+      Mh[h] = -INFINITY;
+      Lh[h] = 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < kEl; ++i) A[i] = 0.f;
+    for (int ct = fc; ct <= lc; ++ct) {
+      const float* pp = partial_of(ct, pair);
+      float a[kEl], fo[HPK], fn[HPK];
+#pragma unroll
+      for (int i = 0; i < kEl; ++i) a[i] = __ldcg(pp + 2 * HPK + lane + 32 * i);
+#pragma unroll
+      for (int h = 0; h < HPK; ++h) {
+        const float m = __ldcg(pp + h), l = __ldcg(pp + HPK + h);
+        const float Mn = fmaxf(Mh[h], m);
+        fo[h] = Mh[h] == -INFINITY ? 0.f : exp2f(Mh[h] - Mn);
+        fn[h] = exp2f(m - Mn);
+        Lh[h] = Lh[h] * fo[h] + l * fn[h];
+        Mh[h] = Mn;
+      }
+#pragma unroll
+      for (int i = 0; i < kEl; ++i) {
+        const int h = (lane + 32 * i) / D;
+        A[i] = A[i] * fo[h] + a[i] * fn[h];
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kEl; ++i) out[lane + 32 * i] = A[i] / Lh[(lane + 32 * i) / D];
+    if (lane == 0) args.tickets[pair] = 0;  // ready for the next call
+  };
+
   // this warp's state as m[HPK], l[HPK], acc[HPK][D] (fp32) at dst
   auto export_state = [&](float* dst) {
     float lw[C::kChunks];
@@ -930,12 +1044,6 @@ decode_kernel(DecodeArgs args, Split sp) {
     const int k = i % C::kItemSlots;
     const int it = itm[k];
     if (it < 0) break;
-    const bool arrived = mbar_wait_bounded(&bars[k], (uint32_t)(i / C::kItemSlots) & 1u);
-    if (!__all_sync(0xffffffffu, arrived)) {
-      timed_out = true;
-      i_stop = i;
-      break;
-    }
     const int pair = pair_of(sp, it), kk = it - pair * sp.ipp;
     if (pair != cur_pair) {
       if (cur_pair >= 0) {
@@ -944,10 +1052,18 @@ decode_kernel(DecodeArgs args, Split sp) {
         if (lane == 0) atomicOr(&s_parked[cur_pair - p_first], 1u << warp);
         w.reset();
       }
-      // the pair's q (global, HPK x D bf16): read by the warp itself, so its
-      // latency hides under the first item's copy
+      // the pair's q (global, HPK x D bf16), read by the warp itself before it
+      // waits for the item, so that the two latencies overlap
       w.load_pair(args.q + ((long)(pair / args.Hkv) * args.Hq + (long)(pair % args.Hkv) * HPK) * D);
       cur_pair = pair;
+    }
+    // the next item, claimed now: the counter's latency hides under the item
+    const int next = claim();
+    const bool arrived = mbar_wait_bounded(&bars[k], (uint32_t)(i / C::kItemSlots) & 1u);
+    if (!__all_sync(0xffffffffu, arrived)) {
+      timed_out = true;
+      i_stop = i;
+      break;
     }
     unsigned char* base = wbase + k * C::kItemBytes;
     if (kk < sp.n2 + sp.n1) {
@@ -956,11 +1072,11 @@ decode_kernel(DecodeArgs args, Split sp) {
       const int t0 = NG * kGroup + kResTok * (kk - sp.n2 - sp.n1);
       w.residual(base, min(kResTok, S - t0));
     }
-    // release the item slot, claim the next item and start its copies
+    // release the item slot and start the next item's copies into it (the only
+    // generic writes to a slot, residual rows zeroed, are fenced where they happen)
     __syncwarp();
-    if (lane == 0) fence_proxy_async();
-    itm[k] = claim();
-    issue(itm[k], k);
+    itm[k] = next;
+    issue(next, k);
   }
   if (timed_out) {
     // record the failure, then give the copies still in flight a bounded chance
@@ -978,14 +1094,30 @@ decode_kernel(DecodeArgs args, Split sp) {
     export_state(reinterpret_cast<float*>(wbase));
     if (lane == 0) s_final[warp] = cur_pair - p_first;
   }
+  constexpr int kPart = HPK * (D + 2);  // floats of a partial: m[HPK], l[HPK], acc[HPK][D]
+  if (n_pairs <= C::kNW) {
+    // ---- every segment is merged by the last warp of its group to finish: no
+    // CTA-wide barrier, so a group's merge overlaps the other groups' items ----
+    const int seg = s_warp_seg[warp] & 0xffff;
+    __syncwarp();
+    __threadfence_block();  // this warp's state and s_final before its count
+    int last = 0;
+    if (lane == 0) last = atomicAdd(&s_done[seg], 1) == s_gsize[seg] - 1;
+    last = __shfl_sync(0xffffffffu, last, 0);
+    allow_successor();
+    if (!last) return;
+    __threadfence_block();
+    merge_segment(seg);
+    return;
+  }
   __threadfence_block();
   __syncthreads();
   allow_successor();
 
-  // ---- merge the warps of each pair (all threads), then write the outputs ----
-  // Pairs held whole by this CTA go to `out`; a pair shared with other CTAs goes
-  // to this CTA's partial, and the last CTA to arrive merges the partials.
-  constexpr int kPart = HPK * (D + 2);  // floats of a partial: m[HPK], l[HPK], acc[HPK][D]
+  // ---- (more segments than warps) merge the warps of each pair (all threads),
+  // then write the outputs.  Pairs held whole by this CTA go to `out`; a pair
+  // shared with other CTAs goes to this CTA's partial, and the last CTA to
+  // arrive merges the partials.
   // merge tables over the (now unused) q slots, for a batch of pairs at once:
   // the kind of each warp's state for pair k (0 none, 1 its final state in its
   // own shared slots, 2 parked in global memory), its (m, l) and factor

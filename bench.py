@@ -35,7 +35,8 @@ METRIC = ("decode-attention tokens/s and achieved HBM GB/s (% of B200 peak) on p
 FALLBACK_HBM_GBS = 6650.0
 DEFAULT_WORKLOAD = "llama3_8b_gqa_8k"
 KERNEL_SOURCES = ["decode_attention_kivi_b200/csrc/kivi_attn.cu",
-                  "decode_attention_kivi_b200/csrc/kivi_layout.cuh"]
+                  "decode_attention_kivi_b200/csrc/kivi_layout.cuh",
+                  "decode_attention_kivi_b200/csrc/kivi_ptx.cuh"]
 
 
 def parse():

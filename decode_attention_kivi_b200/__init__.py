@@ -18,7 +18,8 @@ from ._native import KiviBuffers, KiviConfig, KiviError, KiviSizes, check, lib
 
 __all__ = [
     "KiviCache", "KiviConfig", "KiviError", "make_config",
-    "kivi_required_bytes", "kivi_cache_create", "kivi_cache_destroy", "kivi_cache_length",
+    "kivi_required_bytes", "kivi_record_layout", "kivi_cache_create", "kivi_cache_destroy",
+    "kivi_cache_length",
     "kivi_cache_reset", "kivi_quantize_prefill", "kivi_append_token", "kivi_decode_attention",
     "kivi_check_device_status", "kivi_cache_bytes", "kivi_status_string",
     "kivi_decode_attention_static_scratch", "kivi_static_scratch_status",
@@ -60,6 +61,14 @@ def kivi_required_bytes(cfg: KiviConfig) -> KiviSizes:
     out = KiviSizes()
     check(lib().kivi_required_bytes(ctypes.byref(cfg), ctypes.byref(out)), "kivi_required_bytes")
     return out
+
+
+def kivi_record_layout(cfg: KiviConfig) -> tuple[int, int]:
+    """(bytes of one group record, records per (layer, sequence, kv head))."""
+    rb, ng = ctypes.c_size_t(), ctypes.c_int32()
+    check(lib().kivi_record_layout(ctypes.byref(cfg), ctypes.byref(rb), ctypes.byref(ng)),
+          "kivi_record_layout")
+    return rb.value, ng.value
 
 
 def kivi_cache_create(cfg: KiviConfig, buffers: KiviBuffers) -> int:
@@ -247,10 +256,10 @@ class KiviCache:
 
     # -- views of the packed state (for tests and inspection) --
     def record_bytes(self) -> int:
-        return self.cfg.head_dim * (32 * self.cfg.bits // 4 + 8)
+        return kivi_record_layout(self.cfg)[0]
 
     def ngcap(self) -> int:
-        return max(0, (self.cfg.max_tokens - RESIDUAL) // GROUP_SIZE)
+        return kivi_record_layout(self.cfg)[1]
 
     def records_view(self, layer: int) -> torch.Tensor:
         c = self.cfg

@@ -49,6 +49,8 @@ def lib() -> ctypes.CDLL:
     st = ctypes.c_int
     sig = {
         "kivi_required_bytes": (st, [ctypes.POINTER(KiviConfig), ctypes.POINTER(KiviSizes)]),
+        "kivi_record_layout": (st, [ctypes.POINTER(KiviConfig), ctypes.POINTER(ctypes.c_size_t),
+                                    ctypes.POINTER(I32)]),
         "kivi_cache_create": (st, [ctypes.POINTER(KiviConfig), ctypes.POINTER(KiviBuffers),
                                    ctypes.POINTER(P)]),
         "kivi_cache_destroy": (None, [P]),

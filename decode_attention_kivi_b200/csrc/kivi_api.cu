@@ -123,6 +123,15 @@ kivi_status kivi_required_bytes(const kivi_config* cfg, kivi_sizes* out) {
   return KIVI_OK;
 }
 
+kivi_status kivi_record_layout(const kivi_config* cfg, size_t* rec_bytes,
+                               int32_t* records_per_seq) {
+  const kivi_status st = validate_config(cfg);
+  if (st != KIVI_OK) return st;
+  if (rec_bytes) *rec_bytes = (size_t)record_bytes(cfg);
+  if (records_per_seq) *records_per_seq = kivi::num_groups(cfg->max_tokens);
+  return KIVI_OK;
+}
+
 kivi_status kivi_cache_create(const kivi_config* cfg, const kivi_buffers* bufs,
                               kivi_cache** out) {
   if (!out || !bufs) return KIVI_ERR_INVALID_ARG;

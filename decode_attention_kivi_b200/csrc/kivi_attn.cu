@@ -85,7 +85,7 @@ constexpr int kSmemBudget = 227 * 1024;
 #define KIVI_ITEM_SLOTS 2
 #endif
 #ifndef KIVI_MAX_WARPS
-#define KIVI_MAX_WARPS 16
+#define KIVI_MAX_WARPS 12  // measured: 12 warps per SM beat 16 (and 14, 11, 10)
 #endif
 
 // ---------------------------------------------------------------------------
@@ -205,9 +205,11 @@ struct Cfg {
   static_assert(kStateFloats * 4 <= kItemSlots * kItemBytes, "a warp's final state fits its item slots");
   static constexpr int kMinSlots = 4;
   static constexpr int kFixed = 2048;                     // mbarriers, counters, masks
+  // warps per CTA: a multiple of 4, so that the four schedulers of an SM hold
+  // the same number of warps
   static constexpr int kNW =
       cmin_i(HPK > 4 ? cmin_i(8, KIVI_MAX_WARPS) : KIVI_MAX_WARPS,
-             (kSmemBudget - kFixed - kMinSlots * kSlotBytes) / kWarpBytes);
+             (kSmemBudget - kFixed - kMinSlots * kSlotBytes) / kWarpBytes) / 4 * 4;
   static constexpr int kThreads = kNW * 32;
   static constexpr int kSlots =
       cmin_i(64, (kSmemBudget - kFixed - kNW * kWarpBytes) / kSlotBytes);

@@ -135,6 +135,14 @@ typedef struct kivi_cache kivi_cache; /* opaque host handle */
  * Errors: INVALID_ARG (null), UNSUPPORTED (config outside the supported set). */
 kivi_status kivi_required_bytes(const kivi_config* cfg, kivi_sizes* out);
 
+/* Geometry of the records buffer for `cfg`, host only: the bytes of one group
+ * record (G*D*b/4 + 8*D: codes plus fp16 metadata) and the records each
+ * (layer, sequence, kv head) has room for, NGcap = NG(max_tokens) (zero when
+ * max_tokens < R).  Records are ordered [layer][sequence][kv head][NGcap].
+ * Either output may be NULL.  Errors: INVALID_ARG (null cfg), UNSUPPORTED. */
+kivi_status kivi_record_layout(const kivi_config* cfg, size_t* record_bytes,
+                               int32_t* records_per_seq);
+
 /* Creates a handle over caller-owned buffers; every layer starts empty (S = 0).
  * Zeroes the device status word in `workspace` with a synchronous cudaMemset.
  * Errors: INVALID_ARG, UNSUPPORTED, BUFFER_TOO_SMALL, CUDA. */

@@ -165,3 +165,15 @@ def test_fake_quant_keys_validation(lib):
     assert N.STATUS[lib.kivi_fake_quant_keys(fake, 32, 96, 2, 0, fake, None)] == \
         "KIVI_ERR_UNSUPPORTED"
     assert lib.kivi_fake_quant_keys(fake, 0, 128, 2, 1, fake, None) == 0  # nothing to do
+
+
+def test_record_layout_query(lib):
+    """The binding's record views take the record size and count from the library."""
+    import oracle as O2
+    for D, bits, mt in [(128, 2, 8192 + 64), (128, 4, 300), (64, 2, 100)]:
+        c = cfg(head_dim=D, bits=bits, max_tokens=mt)
+        rb, ng = ctypes.c_size_t(), ctypes.c_int32()
+        assert lib.kivi_record_layout(ctypes.byref(c), ctypes.byref(rb), ctypes.byref(ng)) == 0
+        assert rb.value == O2.record_bytes(D, bits)
+        assert ng.value == O2.num_groups(mt)
+    assert N.STATUS[lib.kivi_record_layout(None, None, None)] == "KIVI_ERR_INVALID_ARG"

@@ -66,22 +66,19 @@ long partial_bytes(const kivi_config* c) {
   return kivi::decode_partial_bytes(c->head_dim, c->num_q_heads / c->num_kv_heads);
 }
 
-// Bytes before the partials: status header, tickets, parked warp states.
+// Bytes before the partials: status header, tickets.
 long fixed_workspace_bytes(const kivi_config* c) {
   const long pairs = (long)c->batch * c->num_kv_heads;
-  return kivi::kWsHeader + kivi::ws_tickets_bytes(pairs) +
-         kivi::decode_parks_bytes(c->head_dim, c->num_q_heads / c->num_kv_heads, pairs);
+  return kivi::kWsHeader + kivi::ws_tickets_bytes(pairs);
 }
 
 // Points the decode arguments at a workspace of `bytes` bytes: status header,
-// tickets, parked warp states, then as many CTAs' partials as fit.
+// tickets, then as many CTAs' partials as fit.
 void bind_workspace(kivi::DecodeArgs& a, const kivi_config* c, void* ws, size_t bytes) {
-  const long pairs = (long)c->batch * c->num_kv_heads;
   uint8_t* base = static_cast<uint8_t*>(ws);
   const long fixed = fixed_workspace_bytes(c);
   a.status = reinterpret_cast<uint32_t*>(base);
   a.tickets = reinterpret_cast<int*>(base + kivi::kWsHeader);
-  a.parks = reinterpret_cast<float*>(base + kivi::kWsHeader + kivi::ws_tickets_bytes(pairs));
   a.partials = reinterpret_cast<float*>(base + fixed);
   const long room = (long)bytes - fixed;
   a.max_ctas = room > 0 ? (int)(room / partial_bytes(c)) : 0;
@@ -489,7 +486,7 @@ extern "C" kivi_status kivi_decode_attention_static_scratch(
   const long pairs = (long)cfg->batch * cfg->num_kv_heads;
   const int hpk = cfg->num_q_heads / cfg->num_kv_heads;
 
-  // the fixed part (status word, tickets, parked states) must fit before any device work
+  // the fixed part (status word, tickets) must fit before any device work
   const long fixed = fixed_workspace_bytes(cfg);
   if (fixed + partial_bytes(cfg) > (long)KIVI_STATIC_SCRATCH_BYTES) return KIVI_ERR_SCRATCH_LIMIT;
 

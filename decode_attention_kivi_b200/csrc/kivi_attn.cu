@@ -17,11 +17,11 @@
 // the segment's counter, so warps that run ahead take more.  Each warp streams
 // its items into its own two-item shared-memory ring with cp.async.bulk on
 // mbarriers and keeps one online-softmax state.  A warp that has to move to
-// another pair (only when a CTA holds more segments than warps) parks its state
-// in its own global slot, without a lock.  At the end the last warp of each
-// segment's group to finish merges the group's final states on its own (no
-// CTA-wide barrier, so it overlaps the other groups' items); with more segments
-// than warps, all threads merge the final and parked states after one barrier.
+// another pair (only when a CTA holds more segments than warps; then every pair
+// of the CTA belongs to one warp) finishes the pair it leaves from its
+// registers.  At the end the last warp of each segment's group to finish merges
+// the group's final states on its own (no CTA-wide barrier, so it overlaps the
+// other groups' items).
 // A pair held whole goes to the output; for a pair shared with other CTAs the
 // CTA writes a partial, and the last CTA to arrive (a ticket per pair) merges
 // the partials into the output.
@@ -223,13 +223,6 @@ struct Cfg {
   static constexpr int kCostG1 = kRec / 512 + 1;
   static constexpr int kCostR = kResTok * D * 4 / 512 + 1;
 };
-
-// Parked warp states: one slot per (pair, warp) of up to kParkWarps warps, each
-// state m[HPK], l[HPK], acc[HPK][D] in fp32, padded to whole 128-byte lines.
-constexpr int kParkWarps = 16;
-__host__ __device__ constexpr long park_stride_floats(int D, int hpk) {
-  return ((long)hpk * (D + 2) * 4 + 127) / 128 * 32;
-}
 
 // ---------------------------------------------------------------------------
 // The split of the items between CTAs
@@ -740,8 +733,7 @@ decode_kernel(DecodeArgs args, Split sp) {
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffFixed) + C::kItemSlots * warp;
   int* s_ctr = reinterpret_cast<int*>(smem + C::kOffFixed + 8 * C::kItemSlots * C::kNW);
   int* s_final = s_ctr + 4;                          // [kNW] pair (local) of each warp's final state
-  unsigned* s_parked = reinterpret_cast<unsigned*>(s_final + C::kNW);  // [kSlots] warp bitmasks
-  int* s_seg_next = reinterpret_cast<int*>(s_parked + C::kSlots);      // [kSlots] claim counters
+  int* s_seg_next = s_final + C::kNW;                                  // [kSlots] claim counters
   int* s_seg_end = s_seg_next + C::kSlots;                             // [kSlots] end items
   int* s_gsize = s_seg_end + C::kSlots + C::kNW;  // [kSlots] warps of each segment (after s_warp_seg)
   int* s_done = s_gsize + C::kSlots;              // [kSlots] warps of each segment that finished
@@ -760,7 +752,6 @@ decode_kernel(DecodeArgs args, Split sp) {
       s_final[warp] = -1;
     }
     for (int k = threadIdx.x; k < n_pairs; k += C::kThreads) {
-      s_parked[k] = 0u;
       s_done[k] = 0;
       s_seg_next[k] = max(it_begin, (p_first + k) * sp.ipp);
       s_seg_end[k] = min(it_end, (p_first + k + 1) * sp.ipp);
@@ -893,6 +884,52 @@ decode_kernel(DecodeArgs args, Split sp) {
   // of them have counted themselves done) and writes the pair's output, or this
   // CTA's partial and the pair's ticket; the CTA that takes the last ticket of a
   // shared pair merges the pair's partials.
+  // After this warp wrote its CTA's partial of a shared pair: takes the pair's
+  // ticket, and if this CTA is the last of the pair's CTAs to arrive, merges the
+  // partials (online, CTA by CTA, all of a lane's elements in flight) into out.
+  auto ticket_and_combine = [&](int pair, int fc, int lc, float* out) {
+    constexpr int kEl = HPK * D / 32;
+    __threadfence();  // the partial before the ticket
+    __syncwarp();
+    int is_last = 0;
+    if (lane == 0) is_last = atomicAdd(&args.tickets[pair], 1) == lc - fc;
+    is_last = __shfl_sync(0xffffffffu, is_last, 0);
+    if (!is_last) return;
+    __threadfence();
+    float A[kEl];
+    // the pair's partials, CTA by CTA (online), all of a lane's elements at once
+    float Mh[HPK], Lh[HPK];
+#pragma unroll
+    for (int h = 0; h < HPK; ++h) {
+      Mh[h] = -INFINITY;
+      Lh[h] = 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < kEl; ++i) A[i] = 0.f;
+    for (int ct = fc; ct <= lc; ++ct) {
+      const float* pp = partial_of(ct, pair);
+      float a[kEl], fo[HPK], fn[HPK];
+#pragma unroll
+      for (int i = 0; i < kEl; ++i) a[i] = __ldcg(pp + 2 * HPK + lane + 32 * i);
+#pragma unroll
+      for (int h = 0; h < HPK; ++h) {
+        const float m = __ldcg(pp + h), l = __ldcg(pp + HPK + h);
+        const float Mn = fmaxf(Mh[h], m);
+        fo[h] = Mh[h] == -INFINITY ? 0.f : exp2f(Mh[h] - Mn);
+        fn[h] = exp2f(m - Mn);
+        Lh[h] = Lh[h] * fo[h] + l * fn[h];
+        Mh[h] = Mn;
+      }
+#pragma unroll
+      for (int i = 0; i < kEl; ++i) {
+        const int h = (lane + 32 * i) / D;
+        A[i] = A[i] * fo[h] + a[i] * fn[h];
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kEl; ++i) out[lane + 32 * i] = A[i] / Lh[(lane + 32 * i) / D];
+    if (lane == 0) args.tickets[pair] = 0;  // ready for the next call
+  };
   auto merge_segment = [&](int seg) {
     constexpr int kEl = HPK * D / 32;  // elements of a state per lane: e = lane + 32 i
     const int pair = p_first + seg;
@@ -949,45 +986,7 @@ decode_kernel(DecodeArgs args, Split sp) {
       part[lane] = s_M[lane];
       part[HPK + lane] = s_M[HPK + lane];
     }
-    __threadfence();  // the partial before the ticket
-    __syncwarp();
-    int is_last = 0;
-    if (lane == 0) is_last = atomicAdd(&args.tickets[pair], 1) == lc - fc;
-    is_last = __shfl_sync(0xffffffffu, is_last, 0);
-    if (!is_last) return;
-    __threadfence();
-    // the pair's partials, CTA by CTA (online), all of a lane's elements at once
-    float Mh[HPK], Lh[HPK];
-#pragma unroll
-    for (int h = 0; h < HPK; ++h) {
-      Mh[h] = -INFINITY;
-      Lh[h] = 0.f;
-    }
-#pragma unroll
-    for (int i = 0; i < kEl; ++i) A[i] = 0.f;
-    for (int ct = fc; ct <= lc; ++ct) {
-      const float* pp = partial_of(ct, pair);
-      float a[kEl], fo[HPK], fn[HPK];
-#pragma unroll
-      for (int i = 0; i < kEl; ++i) a[i] = __ldcg(pp + 2 * HPK + lane + 32 * i);
-#pragma unroll
-      for (int h = 0; h < HPK; ++h) {
-        const float m = __ldcg(pp + h), l = __ldcg(pp + HPK + h);
-        const float Mn = fmaxf(Mh[h], m);
-        fo[h] = Mh[h] == -INFINITY ? 0.f : exp2f(Mh[h] - Mn);
-        fn[h] = exp2f(m - Mn);
-        Lh[h] = Lh[h] * fo[h] + l * fn[h];
-        Mh[h] = Mn;
-      }
-#pragma unroll
-      for (int i = 0; i < kEl; ++i) {
-        const int h = (lane + 32 * i) / D;
-        A[i] = A[i] * fo[h] + a[i] * fn[h];
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < kEl; ++i) out[lane + 32 * i] = A[i] / Lh[(lane + 32 * i) / D];
-    if (lane == 0) args.tickets[pair] = 0;  // ready for the next call
+    ticket_and_combine(pair, fc, lc, out);
   };
 
   // this warp's state as m[HPK], l[HPK], acc[HPK][D] (fp32) at dst
@@ -1037,10 +1036,81 @@ decode_kernel(DecodeArgs args, Split sp) {
     }
   };
 
+  // out = acc / l of this warp's state for the HPK heads of a pair (out: the
+  // pair's first head, HPK x D fp32), the same elements as export_state
+  auto export_output = [&](float* out) {
+    float lw[C::kChunks];
+#pragma unroll
+    for (int c = 0; c < C::kChunks; ++c) {
+      float l = w.l_run[c];
+      l += __shfl_xor_sync(0xffffffffu, l, 4);
+      l += __shfl_xor_sync(0xffffffffu, l, 8);
+      l += __shfl_xor_sync(0xffffffffu, l, 16);
+      lw[c] = l;  // head 4c + tig
+    }
+    float inv[2];  // 1 / l of heads 2tig + e (lanes tig < 2 only, for <= 4 heads)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int h = (2 * w.tig + e) & 7;
+      const int src = (lane & ~3) | (h & 3);
+      float l = __shfl_sync(0xffffffffu, lw[0], src);
+      if constexpr (C::kChunks == 2) {
+        const float l1 = __shfl_sync(0xffffffffu, lw[C::kChunks - 1], src);
+        l = h >= 4 ? l1 : l;
+      }
+      inv[e] = 1.f / l;
+    }
+    float vm[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) vm[r] = w.vmacc[r];
+    if constexpr (C::kLoCols) {
+#pragma unroll
+      for (int r = 0; r < 4; ++r) vm[r] -= __shfl_xor_sync(0xffffffffu, vm[r], 2);
+    }
+    float vb[W::kBlocks][2];
+#pragma unroll
+    for (int j = 0; j < W::kBlocks; ++j) {
+      vb[j][0] = __shfl_sync(0xffffffffu, vm[0], 4 * j + w.tig);
+      vb[j][1] = __shfl_sync(0xffffffffu, vm[1], 4 * j + w.tig);
+    }
+    const bool valid_lane = C::kLoCols ? w.tig < 2 : true;
+#pragma unroll
+    for (int mt = 0; mt < W::kMTiles; ++mt) {
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        float x = w.acc[mt][r];
+        if constexpr (C::kLoCols) x -= __shfl_xor_sync(0xffffffffu, x, 2);
+        x = x * (float)(1 << C::kCodeShift) + vb[mt / 2][r & 1];
+        const int h = 2 * w.tig + (r & 1);
+        if (valid_lane && h < HPK) out[h * D + 16 * mt + w.g + 8 * (r >> 1)] = x * inv[r & 1];
+      }
+    }
+  };
+
+  // With more segments than warps every pair of the CTA belongs to one warp:
+  // when the warp leaves it, its state is the CTA's whole result for the pair.
+  // A pair held whole goes straight to out (acc / l from the registers); the
+  // CTA's first or last pair, when shared, goes to the CTA's partial and its
+  // ticket.
+  auto finish_pair = [&](int pair) {
+    const int fc = cta_of_item(sp, pair * sp.ipp), lc = cta_of_item(sp, pair * sp.ipp + sp.ipp - 1);
+    const int b = pair / args.Hkv, kvh = pair % args.Hkv;
+    float* out = args.out + ((long)b * args.Hq + (long)kvh * HPK) * D;
+    if (fc != lc) {
+      if (cta >= args.max_ctas) {  // the host's split rules exclude this
+        if (lane == 0) atomicOr(args.status, kStatusBadSplit);
+        return;
+      }
+      export_state(partial_of(cta, pair));
+      ticket_and_combine(pair, fc, lc, out);
+      return;
+    }
+    export_output(out);
+  };
+
   int cur_pair = -1;
   bool timed_out = false;
   int i_stop = 0;
-  const long park_stride = park_stride_floats(D, HPK);
 
   for (int i = 0;; ++i) {
     const int k = i % C::kItemSlots;
@@ -1048,10 +1118,8 @@ decode_kernel(DecodeArgs args, Split sp) {
     if (it < 0) break;
     const int pair = pair_of(sp, it), kk = it - pair * sp.ipp;
     if (pair != cur_pair) {
-      if (cur_pair >= 0) {
-        // park the state of the pair this warp leaves: its own slot, no lock
-        export_state(args.parks + ((long)cur_pair * kParkWarps + warp) * park_stride);
-        if (lane == 0) atomicOr(&s_parked[cur_pair - p_first], 1u << warp);
+      if (cur_pair >= 0) {  // (only with more segments than warps)
+        finish_pair(cur_pair);
         w.reset();
       }
       // the pair's q (global, HPK x D bf16), read by the warp itself before it
@@ -1091,13 +1159,12 @@ decode_kernel(DecodeArgs args, Split sp) {
     }
     __syncwarp();
   }
-  // the final state goes to this warp's own item slots (no copy is in flight any more)
-  if (cur_pair >= 0) {
-    export_state(reinterpret_cast<float*>(wbase));
-    if (lane == 0) s_final[warp] = cur_pair - p_first;
-  }
-  constexpr int kPart = HPK * (D + 2);  // floats of a partial: m[HPK], l[HPK], acc[HPK][D]
   if (n_pairs <= C::kNW) {
+    // the final state goes to this warp's own item slots (no copy is in flight any more)
+    if (cur_pair >= 0) {
+      export_state(reinterpret_cast<float*>(wbase));
+      if (lane == 0) s_final[warp] = cur_pair - p_first;
+    }
     // ---- every segment is merged by the last warp of its group to finish: no
     // CTA-wide barrier, so a group's merge overlaps the other groups' items ----
     const int seg = s_warp_seg[warp] & 0xffff;
@@ -1112,143 +1179,8 @@ decode_kernel(DecodeArgs args, Split sp) {
     merge_segment(seg);
     return;
   }
-  __threadfence_block();
-  __syncthreads();
   allow_successor();
-
-  // ---- (more segments than warps) merge the warps of each pair (all threads),
-  // then write the outputs.  Pairs held whole by this CTA go to `out`; a pair
-  // shared with other CTAs goes to this CTA's partial, and the last CTA to
-  // arrive merges the partials.
-  // merge tables over the (now unused) q slots, for a batch of pairs at once:
-  // the kind of each warp's state for pair k (0 none, 1 its final state in its
-  // own shared slots, 2 parked in global memory), its (m, l) and factor
-  // 2^(m - M) per head, the merged M and L, and where the result goes
-  const int nw = C::kNW;
-  constexpr int kTableBytes = C::kNW * 4 + C::kNW * HPK * 12 + HPK * 8 + 16;
-  constexpr int kBatch = C::kSlots * C::kSlotBytes / kTableBytes;
-  static_assert(kBatch >= 1, "merge tables of one pair fit the q slots");
-  bool wrote_partial = false;
-  for (int k0 = 0; k0 < n_pairs; k0 += kBatch) {
-    const int nb = min(kBatch, n_pairs - k0);
-    int* s_kind = reinterpret_cast<int*>(smem + C::kOffSlots);  // [nb][kNW]
-    float* s_m = reinterpret_cast<float*>(s_kind + nb * nw);      // [nb][kNW][HPK]
-    float* s_l = s_m + nb * nw * HPK;
-    float* s_f = s_l + nb * nw * HPK;
-    float* s_ML = s_f + nb * nw * HPK;                              // [nb][2][HPK]
-    int* s_dest = reinterpret_cast<int*>(s_ML + nb * 2 * HPK);      // [nb]: -1 out, else side
-    int* s_anypark = s_dest + nb;                                   // [nb]
-    for (int t = threadIdx.x; t < nb * nw; t += C::kThreads) {
-      const int k = k0 + t / nw, ww = t % nw;
-      s_kind[t] = s_final[ww] == k ? 1 : ((s_parked[k] >> ww & 1u) ? 2 : 0);
-    }
-    __syncthreads();
-    for (int t = threadIdx.x; t < nb * nw * HPK; t += C::kThreads) {  // every state header
-      const int kw = t / HPK, h = t % HPK, ww = kw % nw;
-      const int kind = s_kind[kw];
-      const float* src = kind == 1 ? reinterpret_cast<const float*>(smem + ww * C::kWarpBytes)
-                                   : args.parks + ((long)(p_first + k0 + kw / nw) * kParkWarps + ww) * park_stride;
-      s_m[t] = kind ? src[h] : -INFINITY;
-      s_l[t] = kind ? src[HPK + h] : 0.f;
-    }
-    __syncthreads();
-    for (int t = threadIdx.x; t < nb * HPK; t += C::kThreads) {
-      const int kb = t / HPK, h = t % HPK;
-      float M = -INFINITY;
-      for (int ww = 0; ww < nw; ++ww) M = fmaxf(M, s_m[(kb * nw + ww) * HPK + h]);
-      float L = 0.f;
-      for (int ww = 0; ww < nw; ++ww) {
-        const int i = (kb * nw + ww) * HPK + h;
-        const float f = s_m[i] == -INFINITY ? 0.f : exp2f(s_m[i] - M);
-        L += s_l[i] * f;
-        s_f[i] = f;
-      }
-      s_ML[kb * 2 * HPK + h] = M;
-      s_ML[kb * 2 * HPK + HPK + h] = L;
-      if (h == 0) {
-        const int pair = p_first + k0 + kb;
-        const int fc = cta_of_item(sp, pair * sp.ipp);
-        const int lc = cta_of_item(sp, pair * sp.ipp + sp.ipp - 1);
-        s_dest[kb] = fc == lc ? -1 : (pair == p_first ? 0 : 1);
-        int any = 0;
-        for (int ww = 0; ww < nw; ++ww) any |= s_kind[kb * nw + ww] == 2;
-        s_anypark[kb] = any;
-      }
-    }
-    __syncthreads();
-    for (int t = threadIdx.x; t < nb * HPK * D; t += C::kThreads) {
-      const int kb = t / (HPK * D), e = t % (HPK * D), h = e / D;
-      const int pair = p_first + k0 + kb;
-      const float* f = s_f + kb * nw * HPK + h;
-      float A = 0.f;
-#pragma unroll
-      for (int ww = 0; ww < C::kNW; ++ww)  // final states in the warps' own slots
-        if (s_kind[kb * nw + ww] == 1)
-          A = fmaf(f[ww * HPK], reinterpret_cast<const float*>(smem + ww * C::kWarpBytes)[2 * HPK + e], A);
-      if (s_anypark[kb]) {  // parked states (a warp that swept several segments)
-        for (int ww = 0; ww < nw; ++ww)
-          if (s_kind[kb * nw + ww] == 2)
-            A = fmaf(f[ww * HPK], args.parks[((long)pair * kParkWarps + ww) * park_stride + 2 * HPK + e], A);
-      }
-      const int dest = s_dest[kb];
-      if (dest < 0) {
-        const int b = pair / args.Hkv, kvh = pair % args.Hkv;
-        args.out[((long)b * args.Hq + (long)kvh * HPK) * D + e] = A / s_ML[kb * 2 * HPK + HPK + h];
-      } else if (cta < args.max_ctas) {
-        float* part = args.partials + ((long)cta * 2 + dest) * kPart;
-        part[2 * HPK + e] = A;
-        if (e % D == 0) {
-          part[h] = s_ML[kb * 2 * HPK + h];
-          part[HPK + h] = s_ML[kb * 2 * HPK + HPK + h];
-        }
-        wrote_partial = true;
-      }
-    }
-    __syncthreads();  // the tables are rebuilt for the next batch
-  }
-  if (__syncthreads_or(wrote_partial)) __threadfence();
-  // tickets of the shared pairs (only the first and the last pair of a CTA can
-  // be shared): thread 0 takes them; the CTA that arrives last at a pair merges
-  // that pair's partials with all its threads
-  int* s_last = reinterpret_cast<int*>(smem + C::kOffSlots);  // [2]: pair this CTA completes, or -1
-  if (threadIdx.x < 2) s_last[threadIdx.x] = -1;
-  __syncthreads();
-  if (threadIdx.x < 2 && cta < args.max_ctas) {  // both tickets at once
-    const int side = threadIdx.x;
-    const int pair = side == 0 ? p_first : p_last;
-    if (side == 0 || p_last != p_first) {
-      const int fc = cta_of_item(sp, pair * sp.ipp), lc = cta_of_item(sp, pair * sp.ipp + sp.ipp - 1);
-      if (fc != lc && atomicAdd(&args.tickets[pair], 1) == lc - fc) s_last[side] = pair;
-    }
-  }
-  if (threadIdx.x == 0 && cta >= args.max_ctas) atomicOr(args.status, kStatusBadSplit);
-  __syncthreads();
-  for (int side = 0; side < 2; ++side) {
-    const int pair = s_last[side];
-    if (pair < 0) continue;
-    __threadfence();
-    const int fc = cta_of_item(sp, pair * sp.ipp), lc = cta_of_item(sp, pair * sp.ipp + sp.ipp - 1);
-    const int b = pair / args.Hkv, kvh = pair % args.Hkv;
-    float* out = args.out + ((long)b * args.Hq + (long)kvh * HPK) * D;
-    // partial of CTA ct: side 0 if the pair is ct's first pair (only fc can hold
-    // it as its last pair)
-    for (int e = threadIdx.x; e < HPK * D; e += C::kThreads) {
-      const int h = e / D;
-      float M = -INFINITY, L = 0.f, A = 0.f;  // online merge: the loads of all parts overlap
-#pragma unroll 4
-      for (int ct = fc; ct <= lc; ++ct) {
-        const float* pp = args.partials + ((long)ct * 2 + (ct == fc && pair != cta_first_item(sp, ct) / sp.ipp ? 1 : 0)) * kPart;
-        const float m = __ldcg(pp + h), l = __ldcg(pp + HPK + h), a = __ldcg(pp + 2 * HPK + e);
-        const float Mn = fmaxf(M, m);
-        const float fo = M == -INFINITY ? 0.f : exp2f(M - Mn), fn = exp2f(m - Mn);
-        L = L * fo + l * fn;
-        A = A * fo + a * fn;
-        M = Mn;
-      }
-      out[e] = A / L;
-    }
-    if (threadIdx.x == 0) args.tickets[pair] = 0;  // ready for the next call
-  }
+  if (cur_pair >= 0) finish_pair(cur_pair);  // the warp's last pair (more segments than warps)
 }
 
 // ---------------------------------------------------------------------------
@@ -1379,16 +1311,11 @@ int decode_grid_ctas(int D, int bits, int hpk, long pairs, int S, int num_sms) {
   return 0;
 }
 
-long decode_parks_bytes(int D, int hpk, long pairs) {
-  return pairs * kParkWarps * park_stride_floats(D, hpk) * (long)sizeof(float);
-}
-
 long decode_partial_bytes(int D, int hpk) { return 2L * hpk * (D + 2) * (long)sizeof(float); }
 
 long decode_workspace_bytes(int D, int bits, int hpk, long pairs) {
   const long ctas = decode_max_ctas(D, bits, hpk, pairs);
-  return kWsHeader + ws_tickets_bytes(pairs) + decode_parks_bytes(D, hpk, pairs) +
-         ctas * decode_partial_bytes(D, hpk);
+  return kWsHeader + ws_tickets_bytes(pairs) + ctas * decode_partial_bytes(D, hpk);
 }
 
 cudaError_t launch_decode(int D, int bits, const DecodeArgs& a, cudaStream_t stream) {

@@ -35,7 +35,6 @@ struct DecodeArgs {
   float* out;                    // [B][Hq][D]
   uint32_t* status;              // device status word
   int* tickets;                  // one per (sequence, kv head); zero between calls
-  float* parks;                  // [B*Hkv][16 warps] parked warp states
   float* partials;               // [max_ctas][2][Hq/Hkv][D + 2] split partials
   int max_ctas;                  // capacity of `partials` in CTAs
   int B, Hkv, Hq, S, ngcap;
@@ -45,11 +44,10 @@ struct DecodeArgs {
 };
 
 // Workspace of the decode kernel for `pairs` (sequence, kv head) pairs, in
-// order: status header, tickets, parked warp states (parks_bytes), then the
+// order: status header, tickets, then the
 // per-CTA partials (partial_bytes each) of the largest grid it uses
 // (decode_max_ctas).  Host-only arithmetic; no device is queried.
 int decode_max_ctas(int D, int bits, int hpk, long pairs);
-long decode_parks_bytes(int D, int hpk, long pairs);
 long decode_partial_bytes(int D, int hpk);
 // CTAs the decode kernel launches for this shape on a device with num_sms SMs
 // (0 for an unsupported shape).

@@ -57,14 +57,11 @@ def test_required_bytes_layout(lib):
     ngcap = O.num_groups(c.max_tokens)
     assert s.records_bytes == 32 * 16 * 8 * ngcap * 3072
     assert s.resid_k_bytes == s.resid_v_bytes == 32 * 16 * 8 * 160 * 128 * 2
-    # status header, one ticket per (sequence, kv head) rounded to 256 bytes, parked
-    # warp states, and two (m, l, acc) partials of the 4 query heads of a kv head per
-    # CTA, for 256 CTAs
+    # status header, one ticket per (sequence, kv head) rounded to 256 bytes, and two
+    # (m, l, acc) partials of the 4 query heads of a kv head per CTA, for 256 CTAs
     pairs = 16 * 8
     tickets = (4 * pairs + 255) // 256 * 256
-    # parked warp states: 16 per pair, each m, l and acc of 4 heads padded to 128-byte lines
-    park = (4 * 130 * 4 + 127) // 128 * 128
-    assert s.workspace_bytes == 256 + tickets + pairs * 16 * park + 256 * 2 * 4 * (128 + 2) * 4
+    assert s.workspace_bytes == 256 + tickets + 256 * 2 * 4 * (128 + 2) * 4
 
 
 @pytest.mark.parametrize("field,value,code", [

@@ -84,6 +84,16 @@ def test_many_splits(kivi):
     _run_small(kivi, B=1, Hkv=1, Hq=4, D=128, bits=2, S0=8192, steps=1, seed=91)
 
 
+@pytest.mark.parametrize("B,Hkv,Hq,D,bits,S0", [(128, 16, 16, 64, 2, 300), (80, 16, 128, 64, 4, 200),
+                                                (128, 16, 64, 128, 2, 161)])
+def test_more_pairs_than_warps_per_cta(kivi, B, Hkv, Hq, D, bits, S0):
+    """Thousands of short (sequence, kv head) pairs: every CTA holds more pairs than warps,
+    so each warp sweeps whole pairs and finishes each from its registers (the output, or
+    the CTA's partial and ticket for its first and last pair)."""
+    _run_small(kivi, B=B, Hkv=Hkv, Hq=Hq, D=D, bits=bits, S0=S0, steps=2, seed=B + Hq + S0,
+               check_each=False)
+
+
 def test_decode_without_prefill(kivi):
     """Append-only growth from an empty layer through the first flush."""
     _run_small(kivi, B=1, Hkv=1, Hq=1, D=128, bits=2, S0=0, steps=165, seed=5, check_each=False)

@@ -33,6 +33,7 @@ import synth  # noqa: E402
 
 METRIC = ("decode-attention tokens/s and achieved HBM GB/s (% of B200 peak) on packed cache")
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 DEFAULT_WORKLOAD = "llama3_8b_gqa_8k"
 KERNEL_SOURCES = ["decode_attention_kivi_b200/csrc/kivi_attn.cu",
                   "decode_attention_kivi_b200/csrc/kivi_layout.cuh",
@@ -51,11 +52,13 @@ def parse():
                    help="override the workload's layer count (small profiling captures)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
-    p.add_argument("--sweep", choices=["memory-wall", "key-granularity"], default=None,
+    p.add_argument("--sweep", choices=["memory-wall", "key-granularity", "prefill"], default=None,
                    help="memory-wall: decode attention of the 2-bit cache and of a bf16 cache "
                         "over growing batches of the Llama-2-13B MHA 4K shape, until a cache "
                         "no longer fits (one JSON line)")
     p.add_argument("--sweep-batches", default="16,32,48,53,64,96,128,160,192,224,240,256")
+    p.add_argument("--prefill-batches", default="1,4,16",
+                   help="prefill sweep: batches of 8K prompts of one Llama-3-8B GQA layer")
     return p.parse_args()
 
 
@@ -134,6 +137,16 @@ def percentiles(xs) -> dict:
     pick = lambda f: ys[min(len(ys) - 1, max(0, int(round(f * (len(ys) - 1)))))]
     return {"median": statistics.median(ys), "p10": pick(0.10), "p90": pick(0.90),
             "mean": sum(ys) / len(ys), "n": len(ys)}
+
+
+def tensor_peak():
+    """Dense bf16 tensor peak (TFLOP/s) for a kernel timed alone: the measured burst."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def hbm_peak():
@@ -776,8 +789,77 @@ def run_key_granularity(args):
                       "data": "synthetic (seeded)"}), flush=True)
 
 
+# ---------------------------------------------------------------------------
+# Prefill: causal attention on the tensor cores, with and without the fused quantize
+# ---------------------------------------------------------------------------
+
+def causal_attention_flops(B, Hq, D, S) -> int:
+    """Multiply-adds x 2 of the causal attention's two products: position i takes
+    i + 1 keys, so sum_i (i + 1) = S (S + 1) / 2 dot products of length D each."""
+    return 2 * 2 * B * Hq * D * (S * (S + 1) // 2)
+
+
+def run_prefill(args):
+    """One Llama-3-8B GQA layer's 8K prompt: the causal attention alone, the same
+    with the prompt quantized into the cache in its epilogue, and the separate
+    quantize kernels, each timed with CUDA events (median of 10 calls)."""
+    import decode_attention_kivi_b200 as K
+
+    device = torch.device("cuda", torch.cuda.current_device())
+    w0 = synth.WORKLOADS["llama3_8b_gqa_8k"]
+    S = w0.context
+    peak, peak_kind = tensor_peak()
+    rows = []
+    for B in [int(x) for x in args.prefill_batches.split(",")]:
+        w = w0.with_batch(B)
+        q = synth.prompt_query(w, 0, device=device)
+        k, v = synth.prefill_kv(w, 0, device=device)
+        out = torch.empty(q.shape, dtype=torch.float32, device=device)
+        status = torch.zeros(1, dtype=torch.int32, device=device)
+        cache = K.KiviCache(batch=B, num_layers=1, num_kv_heads=w.num_kv_heads,
+                            num_q_heads=w.num_q_heads, head_dim=w.head_dim, bits=w.bits,
+                            max_tokens=S, device=device)
+
+        def fused(_):
+            cache.reset(0)
+            cache.prefill_attention(0, q, k, v, out)
+
+        def separate_quantize(_):
+            cache.reset(0)
+            cache.prefill(0, k, v)
+
+        ms_attn = _time_layers(lambda _: K.kivi_causal_attention(q, k, v, out, status=status), 1)
+        ms_fused = _time_layers(fused, 1)
+        ms_quant = _time_layers(separate_quantize, 1)
+        assert cache.check_device_status() == 0 and int(status.item()) == 0
+        cache.close()
+        flops = causal_attention_flops(B, w.num_q_heads, w.head_dim, S)
+        tflops = flops / (ms_attn * 1e-3) / 1e12
+        rows.append({"batch": B, "prompt": S, "attention_ms": ms_attn,
+                     "attention_tflops": tflops, "frac_of_peak": tflops / peak,
+                     "fused_prefill_ms": ms_fused,
+                     "fused_tflops": flops / (ms_fused * 1e-3) / 1e12,
+                     "separate_quantize_ms": ms_quant,
+                     "separate_total_ms": ms_attn + ms_quant,
+                     "fused_saves_ms": ms_attn + ms_quant - ms_fused})
+        print(json.dumps(rows[-1]), file=sys.stderr, flush=True)
+        del q, k, v, out
+        torch.cuda.empty_cache()
+    print(json.dumps({
+        "sweep": "prefill", "workload": "llama3_8b_gqa_8k prompt, one layer",
+        "shape": {"kv_heads": w0.num_kv_heads, "q_heads": w0.num_q_heads,
+                  "head_dim": w0.head_dim, "prompt": S, "bits": w0.bits},
+        "metric": "causal prefill attention TFLOP/s (2 x multiply-adds of the causal "
+                  "products) and the time of the fused quantize against the separate kernels",
+        "peak_tflops": peak, "peak_kind": peak_kind, "rows": rows,
+        "data": "synthetic (seeded)", "l2": "inputs larger than L2"}), flush=True)
+
+
 def main():
     args = parse()
+    if args.sweep == "prefill":
+        run_prefill(args)
+        return
     if args.sweep == "memory-wall":
         run_memory_wall(args)
         return

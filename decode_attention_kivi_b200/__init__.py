@@ -20,11 +20,12 @@ __all__ = [
     "KiviCache", "KiviConfig", "KiviError", "make_config",
     "kivi_required_bytes", "kivi_record_layout", "kivi_cache_create", "kivi_cache_destroy",
     "kivi_cache_length",
-    "kivi_cache_reset", "kivi_quantize_prefill", "kivi_append_token", "kivi_decode_attention",
+    "kivi_cache_reset", "kivi_quantize_prefill", "kivi_quantize_prefill_ragged",
+    "kivi_cache_lengths", "kivi_append_token", "kivi_decode_attention",
     "kivi_check_device_status", "kivi_cache_bytes", "kivi_status_string",
     "kivi_decode_attention_static_scratch", "kivi_static_scratch_status",
     "kivi_bf16_workspace_bytes", "kivi_bf16_decode_attention", "kivi_bf16_status",
-    "Bf16Attention", "kivi_fake_quant_keys",
+    "Bf16Attention", "kivi_fake_quant_keys", "kivi_prefill_attention", "kivi_causal_attention",
 ]
 
 GROUP_SIZE = 32
@@ -100,6 +101,21 @@ def kivi_quantize_prefill(handle: int, layer: int, k: torch.Tensor, v: torch.Ten
     check(lib().kivi_quantize_prefill(handle, layer, _ptr(k, torch.bfloat16, "k"),
                                       _ptr(v, torch.bfloat16, "v"), S, _stream(stream)),
           "kivi_quantize_prefill")
+
+
+def kivi_quantize_prefill_ragged(handle: int, layer: int, k: torch.Tensor, v: torch.Tensor,
+                                 lengths, stream=None) -> None:
+    """k, v: bf16 [B][Hkv][S_max][D] on the device; lengths: B ints (tokens per sequence)."""
+    lens = (ctypes.c_int32 * len(lengths))(*[int(x) for x in lengths])
+    check(lib().kivi_quantize_prefill_ragged(handle, layer, _ptr(k, torch.bfloat16, "k"),
+                                             _ptr(v, torch.bfloat16, "v"), k.shape[2], lens,
+                                             _stream(stream)), "kivi_quantize_prefill_ragged")
+
+
+def kivi_cache_lengths(handle: int, layer: int, batch: int) -> list:
+    out = (ctypes.c_int32 * batch)()
+    check(lib().kivi_cache_lengths(handle, layer, out), "kivi_cache_lengths")
+    return list(out)
 
 
 def kivi_append_token(handle: int, layer: int, k_new: torch.Tensor, v_new: torch.Tensor,
@@ -211,6 +227,44 @@ def kivi_fake_quant_keys(k: torch.Tensor, bits: int, per_token: bool,
     return k_hat
 
 
+def _prefill_shapes(q, k, v, out):
+    B, Hq, S, D = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, S, D) or v.shape != k.shape or out.shape != q.shape:
+        raise ValueError("shapes: q and out [B][Hq][S][D], k and v [B][Hkv][S][D]")
+    return B, Hkv, Hq, S, D
+
+
+def kivi_prefill_attention(handle: int, layer: int, q: torch.Tensor, k: torch.Tensor,
+                           v: torch.Tensor, out: torch.Tensor, sm_scale: float = 0.0,
+                           stream=None) -> torch.Tensor:
+    """Causal attention of the prompt (q bf16 [B][Hq][S][D], k, v bf16 [B][Hkv][S][D])
+    into out (fp32 like q), with the prompt quantized into the layer as it goes."""
+    S = _prefill_shapes(q, k, v, out)[3]
+    check(lib().kivi_prefill_attention(handle, layer, _ptr(q, torch.bfloat16, "q"),
+                                       _ptr(k, torch.bfloat16, "k"), _ptr(v, torch.bfloat16, "v"),
+                                       S, _ptr(out, torch.float32, "out"), float(sm_scale),
+                                       _stream(stream)), "kivi_prefill_attention")
+    return out
+
+
+def kivi_causal_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                          out: torch.Tensor | None = None, sm_scale: float = 0.0,
+                          status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Causal attention alone (no cache): q bf16 [B][Hq][S][D], k, v bf16 [B][Hkv][S][D]
+    -> out fp32 [B][Hq][S][D]; status: an optional zeroed int32 device word that a
+    timed-out wait sets."""
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    B, Hkv, Hq, S, D = _prefill_shapes(q, k, v, out)
+    check(lib().kivi_causal_attention(_ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
+                                      _ptr(v, torch.bfloat16, "v"), B, Hkv, Hq, D, S,
+                                      _ptr(out, torch.float32, "out"), float(sm_scale),
+                                      _ptr(status, torch.int32, "status"), _stream(stream)),
+          "kivi_causal_attention")
+    return out
+
+
 class Bf16Attention:
     """Owns the zeroed workspace of kivi_bf16_decode_attention for one shape."""
 
@@ -277,6 +331,18 @@ class KiviCache:
     # -- calls --
     def prefill(self, layer, k, v, stream=None):
         kivi_quantize_prefill(self.handle, layer, k, v, stream=stream)
+
+    def prefill_attention(self, layer, q, k, v, out=None, sm_scale=0.0, stream=None):
+        """Causal attention of the prompt with the prompt quantized into `layer`."""
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        return kivi_prefill_attention(self.handle, layer, q, k, v, out, sm_scale, stream)
+
+    def prefill_ragged(self, layer, k, v, lengths, stream=None):
+        return kivi_quantize_prefill_ragged(self.handle, layer, k, v, lengths, stream)
+
+    def lengths(self, layer) -> list:
+        return kivi_cache_lengths(self.handle, layer, self.cfg.batch)
 
     def append(self, layer, k_new, v_new, stream=None):
         kivi_append_token(self.handle, layer, k_new, v_new, stream=stream)

@@ -58,6 +58,8 @@ def lib() -> ctypes.CDLL:
         "kivi_cache_reset": (st, [P, I32]),
         "kivi_quantize_prefill": (st, [P, I32, P, P, I32, P]),
         "kivi_append_token": (st, [P, I32, P, P, P]),
+        "kivi_quantize_prefill_ragged": (st, [P, I32, P, P, I32, ctypes.POINTER(I32), P]),
+        "kivi_cache_lengths": (st, [P, I32, ctypes.POINTER(I32)]),
         "kivi_decode_attention": (st, [P, I32, P, P, F32, P]),
         "kivi_check_device_status": (st, [P, P, ctypes.POINTER(ctypes.c_uint32)]),
         "kivi_cache_bytes": (st, [ctypes.POINTER(KiviConfig), I32,
@@ -73,6 +75,8 @@ def lib() -> ctypes.CDLL:
                                             ctypes.c_size_t, P]),
         "kivi_bf16_status": (st, [P, I32, I32, P, ctypes.POINTER(ctypes.c_uint32)]),
         "kivi_fake_quant_keys": (st, [P, ctypes.c_int64, I32, I32, I32, P, P]),
+        "kivi_prefill_attention": (st, [P, I32, P, P, P, I32, P, F32, P]),
+        "kivi_causal_attention": (st, [P, P, P, I32, I32, I32, I32, I32, P, F32, P, P]),
     }
     if hasattr(L, "kivi_debug_overstate_copies"):  # debug build only
         sig["kivi_debug_overstate_copies"] = (st, [ctypes.c_uint32])

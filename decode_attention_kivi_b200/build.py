@@ -12,7 +12,8 @@ LIB = os.path.join(PKG, "libkivi.so")
 DEBUG_LIB = os.path.join(PKG, "libkivi_debug.so")
 # debug build: short bounded waits (about 1 ms), copy bounds checks, a test hook
 DEBUG_FLAGS = ["-DKIVI_DEBUG_BUILD", "-DKIVI_DEBUG_BOUNDS", "-DKIVI_DEBUG_WAIT_CYCLES=2000000LL"]
-SOURCES = ["kivi_api.cu", "kivi_quant.cu", "kivi_attn.cu", "kivi_bf16_attn.cu"]
+SOURCES = ["kivi_api.cu", "kivi_quant.cu", "kivi_attn.cu", "kivi_bf16_attn.cu",
+           "kivi_prefill_attn.cu"]
 NVCC_FLAGS = [
     "-O3", "-std=c++17",
     "-gencode", "arch=compute_100a,code=sm_100a",

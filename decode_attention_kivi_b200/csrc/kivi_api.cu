@@ -18,7 +18,10 @@
 struct kivi_cache {
   kivi_config cfg;
   kivi_buffers bufs;
-  std::vector<int32_t> S;  // token count per layer
+  std::vector<int32_t> S;      // token count per layer (the longest sequence's)
+  std::vector<char> ragged;    // layer prefilled with a length per sequence
+  std::vector<std::vector<int32_t>> Sb;  // ragged layers: token count per sequence
+  std::vector<int32_t> steps;  // ragged layers: appends since the prefill
   int ngcap;
   long rec_bytes;
   int num_sms;
@@ -45,6 +48,17 @@ kivi_status validate_config(const kivi_config* c) {
   return KIVI_OK;
 }
 
+// Per-layer prompt lengths of ragged layers ([L][B] int32) at the end of a
+// handle's workspace, after the part the decode kernel uses.
+size_t lens_bytes(const kivi_config* c) {
+  return ((size_t)c->num_layers * c->batch * 4 + 255) / 256 * 256;
+}
+size_t decode_part_bytes(const kivi_config* c) {
+  return (size_t)kivi::decode_workspace_bytes(c->head_dim, c->bits,
+                                              c->num_q_heads / c->num_kv_heads,
+                                              (long)c->batch * c->num_kv_heads);
+}
+
 long record_bytes(const kivi_config* c) {
   return kivi::RecordGeom{c->head_dim, c->bits}.bytes();
 }
@@ -58,7 +72,7 @@ kivi_sizes sizes_of(const kivi_config* c) {
   s.resid_v_bytes = s.resid_k_bytes;
   s.workspace_bytes = (size_t)kivi::decode_workspace_bytes(
       c->head_dim, c->bits, c->num_q_heads / c->num_kv_heads,
-      (long)c->batch * c->num_kv_heads);
+      (long)c->batch * c->num_kv_heads) + lens_bytes(c);
   return s;
 }
 
@@ -107,6 +121,30 @@ __nv_bfloat16* layer_ring(const kivi_cache* h, void* base, int32_t layer) {
 }
 
 kivi_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KIVI_OK : KIVI_ERR_CUDA; }
+
+const int* layer_lens(const kivi_cache* h, int32_t layer) {
+  return reinterpret_cast<const int*>(static_cast<const uint8_t*>(h->bufs.workspace) +
+                                      decode_part_bytes(&h->cfg)) +
+         (size_t)layer * h->cfg.batch;
+}
+
+// The length whose shape the decode split gives every pair.  A ragged layer's
+// pairs take the items of the length with the most items, which need not be the
+// longest: a sequence just short of a flush has more residual rows than a longer
+// one that has just flushed.  Each pair skips the items past its own.
+int32_t decode_shape_len(const kivi_cache* h, int32_t layer) {
+  if (!h->ragged[layer]) return h->S[layer];
+  int32_t best = 0;
+  int best_items = -1;
+  for (const int32_t s : h->Sb[layer]) {
+    const int items = kivi::decode_items(s);
+    if (items > best_items || (items == best_items && s > best)) {
+      best = s;
+      best_items = items;
+    }
+  }
+  return best;
+}
 
 }  // namespace
 
@@ -160,6 +198,9 @@ kivi_status kivi_cache_create(const kivi_config* cfg, const kivi_buffers* bufs,
   h->cfg = *cfg;
   h->bufs = *bufs;
   h->S.assign(cfg->num_layers, 0);
+  h->ragged.assign(cfg->num_layers, 0);
+  h->Sb.assign(cfg->num_layers, std::vector<int32_t>());
+  h->steps.assign(cfg->num_layers, 0);
   h->ngcap = kivi::num_groups(cfg->max_tokens);
   h->rec_bytes = record_bytes(cfg);
   h->num_sms = sms;
@@ -183,6 +224,9 @@ kivi_status kivi_cache_reset(kivi_cache* cache, int32_t layer) {
   kivi_status st = check_layer(cache, layer);
   if (st != KIVI_OK) return st;
   cache->S[layer] = 0;
+  cache->ragged[layer] = 0;
+  cache->Sb[layer].clear();
+  cache->steps[layer] = 0;
   return KIVI_OK;
 }
 
@@ -195,11 +239,12 @@ kivi_status kivi_quantize_prefill(kivi_cache* cache, int32_t layer, const void* 
   if (cache->S[layer] != 0) return KIVI_ERR_STATE;
   if (S > cache->cfg.max_tokens) return KIVI_ERR_CAPACITY;
   if (S > 0) {
-    kivi::PrefillArgs a;
+    kivi::PrefillArgs a{};
     a.k = static_cast<const __nv_bfloat16*>(k);
     a.v = static_cast<const __nv_bfloat16*>(v);
     a.B = cache->cfg.batch;
     a.Hkv = cache->cfg.num_kv_heads;
+    a.lens = nullptr;
     a.S = S;
     a.ng = kivi::num_groups(S);
     a.ngcap = cache->ngcap;
@@ -211,6 +256,139 @@ kivi_status kivi_quantize_prefill(kivi_cache* cache, int32_t layer, const void* 
     if (st != KIVI_OK) return st;
   }
   cache->S[layer] = S;
+  cache->ragged[layer] = 0;
+  cache->Sb[layer].clear();
+  cache->steps[layer] = 0;
+  return KIVI_OK;
+}
+
+namespace {
+kivi_status prefill_attn_shape(int32_t batch, int32_t hkv, int32_t hq, int32_t D, int32_t S) {
+  if (batch < 1 || hkv < 1 || hq < 1 || S < 1) return KIVI_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return KIVI_ERR_UNSUPPORTED;
+  if (hq % hkv != 0) return KIVI_ERR_UNSUPPORTED;
+  if ((long)batch * hq * ((long)S + 128) >= (1L << 31)) return KIVI_ERR_INVALID_ARG;
+  return KIVI_OK;
+}
+bool prefill_ptrs_ok(const void* q, const void* k, const void* v, const void* out) {
+  return q && k && v && out && aligned16(q) && aligned16(k) && aligned16(v) && aligned16(out);
+}
+}  // namespace
+
+kivi_status kivi_prefill_attention(kivi_cache* cache, int32_t layer, const void* q,
+                                   const void* k, const void* v, int32_t S, float* out,
+                                   float sm_scale, void* stream) {
+  kivi_status st = check_layer(cache, layer);
+  if (st != KIVI_OK) return st;
+  const kivi_config& c = cache->cfg;
+  st = prefill_attn_shape(c.batch, c.num_kv_heads, c.num_q_heads, c.head_dim, S);
+  if (st != KIVI_OK) return st;
+  if (!prefill_ptrs_ok(q, k, v, out) || !std::isfinite(sm_scale)) return KIVI_ERR_INVALID_ARG;
+  if (cache->S[layer] != 0) return KIVI_ERR_STATE;
+  if (S > c.max_tokens) return KIVI_ERR_CAPACITY;
+  kivi::PrefillAttnArgs a{};
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k = static_cast<const __nv_bfloat16*>(k);
+  a.v = static_cast<const __nv_bfloat16*>(v);
+  a.out = out;
+  a.status = static_cast<uint32_t*>(cache->bufs.workspace);
+  a.B = c.batch;
+  a.Hkv = c.num_kv_heads;
+  a.Hq = c.num_q_heads;
+  a.S = S;
+  a.sm_scale = sm_scale;
+  a.records = layer_records(cache, layer);
+  a.ring_k = layer_ring(cache, cache->bufs.resid_k, layer);
+  a.ring_v = layer_ring(cache, cache->bufs.resid_v, layer);
+  a.ngcap = cache->ngcap;
+  a.device = cache->device;
+  st = from_cuda(kivi::launch_prefill_attention(c.head_dim, c.bits, a,
+                                                static_cast<cudaStream_t>(stream)));
+  if (st != KIVI_OK) return st;
+  cache->S[layer] = S;
+  cache->ragged[layer] = 0;
+  cache->Sb[layer].clear();
+  cache->steps[layer] = 0;
+  return KIVI_OK;
+}
+
+kivi_status kivi_causal_attention(const void* q, const void* k, const void* v, int32_t batch,
+                                  int32_t num_kv_heads, int32_t num_q_heads, int32_t head_dim,
+                                  int32_t S, float* out, float sm_scale, uint32_t* status,
+                                  void* stream) {
+  kivi_status st = prefill_attn_shape(batch, num_kv_heads, num_q_heads, head_dim, S);
+  if (st != KIVI_OK) return st;
+  if (!prefill_ptrs_ok(q, k, v, out) || !std::isfinite(sm_scale)) return KIVI_ERR_INVALID_ARG;
+  if (status != nullptr && ((uintptr_t)status & 3u) != 0) return KIVI_ERR_INVALID_ARG;
+  int device = 0;
+  if (cudaGetDevice(&device) != cudaSuccess) return KIVI_ERR_CUDA;
+  kivi::PrefillAttnArgs a{};
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k = static_cast<const __nv_bfloat16*>(k);
+  a.v = static_cast<const __nv_bfloat16*>(v);
+  a.out = out;
+  a.status = status;
+  a.B = batch;
+  a.Hkv = num_kv_heads;
+  a.Hq = num_q_heads;
+  a.S = S;
+  a.sm_scale = sm_scale;
+  a.device = device;
+  return from_cuda(kivi::launch_prefill_attention(head_dim, 2, a,
+                                                  static_cast<cudaStream_t>(stream)));
+}
+
+kivi_status kivi_quantize_prefill_ragged(kivi_cache* cache, int32_t layer, const void* k,
+                                         const void* v, int32_t S_max, const int32_t* lengths,
+                                         void* stream) {
+  kivi_status st = check_layer(cache, layer);
+  if (st != KIVI_OK) return st;
+  if (!lengths || S_max < 0) return KIVI_ERR_INVALID_ARG;
+  const int B = cache->cfg.batch;
+  int longest = 0;
+  for (int b = 0; b < B; ++b) {
+    if (lengths[b] < 0 || lengths[b] > S_max) return KIVI_ERR_INVALID_ARG;
+    longest = std::max(longest, (int)lengths[b]);
+  }
+  if (longest > 0 && (!k || !v || !aligned16(k) || !aligned16(v))) return KIVI_ERR_INVALID_ARG;
+  if (cache->S[layer] != 0) return KIVI_ERR_STATE;
+  if (S_max > cache->cfg.max_tokens) return KIVI_ERR_CAPACITY;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* lens = const_cast<int*>(layer_lens(cache, layer));
+  // the lengths go to the workspace once; the kernels derive S_b = lens[b] + steps
+  if (cudaMemcpyAsync(lens, lengths, sizeof(int32_t) * B, cudaMemcpyHostToDevice, s) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return KIVI_ERR_CUDA;
+  if (longest > 0) {
+    kivi::PrefillArgs a{};
+    a.k = static_cast<const __nv_bfloat16*>(k);
+    a.v = static_cast<const __nv_bfloat16*>(v);
+    a.lens = lens;
+    a.B = B;
+    a.Hkv = cache->cfg.num_kv_heads;
+    a.S = S_max;  // the row stride of k and v
+    a.ng = kivi::num_groups(longest);
+    a.ngcap = cache->ngcap;
+    a.records = layer_records(cache, layer);
+    a.ring_k = layer_ring(cache, cache->bufs.resid_k, layer);
+    a.ring_v = layer_ring(cache, cache->bufs.resid_v, layer);
+    st = from_cuda(kivi::launch_prefill(cache->cfg.head_dim, cache->cfg.bits, a, s));
+    if (st != KIVI_OK) return st;
+  }
+  cache->S[layer] = longest;
+  cache->ragged[layer] = 1;
+  cache->Sb[layer].assign(lengths, lengths + B);
+  cache->steps[layer] = 0;
+  return KIVI_OK;
+}
+
+kivi_status kivi_cache_lengths(const kivi_cache* cache, int32_t layer, int32_t* S_out) {
+  kivi_status st = check_layer(cache, layer);
+  if (st != KIVI_OK) return st;
+  if (!S_out) return KIVI_ERR_INVALID_ARG;
+  for (int b = 0; b < cache->cfg.batch; ++b)
+    S_out[b] = cache->ragged[layer] ? cache->Sb[layer][b] : cache->S[layer];
   return KIVI_OK;
 }
 
@@ -219,18 +397,17 @@ kivi_status kivi_append_token(kivi_cache* cache, int32_t layer, const void* k_ne
   kivi_status st = check_layer(cache, layer);
   if (st != KIVI_OK) return st;
   if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return KIVI_ERR_INVALID_ARG;
-  const int S = cache->S[layer];
+  const int S = cache->S[layer];  // the longest sequence's
   if (S + 1 > cache->cfg.max_tokens) return KIVI_ERR_CAPACITY;
-  const int ng = kivi::num_groups(S);
-  kivi::AppendArgs a;
+  kivi::AppendArgs a{};
   a.k_new = static_cast<const __nv_bfloat16*>(k_new);
   a.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  a.lens = cache->ragged[layer] ? layer_lens(cache, layer) : nullptr;
+  a.steps = cache->steps[layer];
   a.B = cache->cfg.batch;
   a.Hkv = cache->cfg.num_kv_heads;
   a.S = S;
   a.ngcap = cache->ngcap;
-  a.flush = (S + 1 - ng * kGroup == kRingSlots) ? 1 : 0;
-  a.ng = ng;
   a.ring_k = layer_ring(cache, cache->bufs.resid_k, layer);
   a.ring_v = layer_ring(cache, cache->bufs.resid_v, layer);
   a.records = layer_records(cache, layer);
@@ -238,6 +415,10 @@ kivi_status kivi_append_token(kivi_cache* cache, int32_t layer, const void* k_ne
                                      static_cast<cudaStream_t>(stream)));
   if (st != KIVI_OK) return st;
   cache->S[layer] = S + 1;
+  if (cache->ragged[layer]) {
+    ++cache->steps[layer];
+    for (int32_t& x : cache->Sb[layer]) ++x;
+  }
   return KIVI_OK;
 }
 
@@ -248,17 +429,22 @@ kivi_status kivi_decode_attention(const kivi_cache* cache, int32_t layer, const 
   if (!q || !out || !aligned16(q) || !aligned16(out)) return KIVI_ERR_INVALID_ARG;
   if (!std::isfinite(sm_scale)) return KIVI_ERR_INVALID_ARG;
   if (cache->S[layer] == 0) return KIVI_ERR_STATE;
-  kivi::DecodeArgs a;
+  if (cache->ragged[layer] &&
+      *std::min_element(cache->Sb[layer].begin(), cache->Sb[layer].end()) == 0)
+    return KIVI_ERR_STATE;  // a sequence without tokens has no attention
+  kivi::DecodeArgs a{};
   a.records = layer_records(cache, layer);
   a.ring_k = layer_ring(cache, cache->bufs.resid_k, layer);
   a.ring_v = layer_ring(cache, cache->bufs.resid_v, layer);
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.out = out;
-  bind_workspace(a, &cache->cfg, cache->bufs.workspace, cache->bufs.sizes.workspace_bytes);
+  bind_workspace(a, &cache->cfg, cache->bufs.workspace, decode_part_bytes(&cache->cfg));
+  a.lens = cache->ragged[layer] ? layer_lens(cache, layer) : nullptr;
+  a.steps = cache->steps[layer];
   a.B = cache->cfg.batch;
   a.Hkv = cache->cfg.num_kv_heads;
   a.Hq = cache->cfg.num_q_heads;
-  a.S = cache->S[layer];
+  a.S = decode_shape_len(cache, layer);
   a.ngcap = cache->ngcap;
   a.sm_scale = sm_scale;
   a.num_sms = cache->num_sms;
@@ -501,7 +687,7 @@ extern "C" kivi_status kivi_decode_attention_static_scratch(
 
   const size_t seqs = (size_t)pairs;
   const long rb = record_bytes(cfg);
-  kivi::DecodeArgs a;
+  kivi::DecodeArgs a{};
   a.records = static_cast<const uint8_t*>(records) + (size_t)layer * seqs * ngcap * rb;
   a.ring_k = static_cast<const __nv_bfloat16*>(resid_k) +
              (size_t)layer * seqs * kRingSlots * cfg->head_dim;

@@ -788,8 +788,21 @@ decode_kernel(DecodeArgs args, Split sp) {
     }
   }
   int seg_cur = 0, seg_hi = 0;  // this warp's segments, read after the barrier below
-  const int NG = sp.NG, S = args.S;
   const long rec_stride = C::kRec;
+  // the items of one pair: n2 record pairs, n1 single records, nr residual items
+  // of its own length S_b (the split is laid out for the longest sequence; the
+  // items of a shorter one past its own count are empty)
+  struct PairShape { int S, NG, n2, n1, nr; };
+  auto pair_shape = [&](int pair) -> PairShape {
+    if (args.lens == nullptr) return PairShape{args.S, sp.NG, sp.n2, sp.n1, sp.nr};
+    PairShape p;
+    p.S = __ldg(args.lens + pair / args.Hkv) + args.steps;
+    p.NG = num_groups(p.S);
+    p.n2 = p.NG / 2;
+    p.n1 = p.NG % 2;
+    p.nr = (p.S - p.NG * kGroup + kResTok - 1) / kResTok;
+    return p;
+  };
   // claims the next item of this warp's segments (warp-uniform; -1 when done)
   auto claim = [&]() -> int {
     while (seg_cur < seg_hi) {
@@ -807,13 +820,18 @@ decode_kernel(DecodeArgs args, Split sp) {
     if (it < 0) return;
     unsigned char* dst = wbase + k * C::kItemBytes;
     const int pair = pair_of(sp, it), kk = it - pair * sp.ipp;
-    if (kk < sp.n2 + sp.n1) {
+    const PairShape ps = pair_shape(pair);
+    if (kk >= ps.n2 + ps.n1 + ps.nr) {  // past this sequence's items: nothing to copy
+      if (lane == 0) mbar_arrive(&bars[k]);
+      return;
+    }
+    if (kk < ps.n2 + ps.n1) {
       if (lane == 0) {
         const int g0 = 2 * kk;
-        const int n_rec = kk < sp.n2 ? 2 : 1;
+        const int n_rec = kk < ps.n2 ? 2 : 1;
         const uint32_t bytes = n_rec * C::kRec;
 #ifdef KIVI_DEBUG_BOUNDS
-        if (pair >= sp.pairs || g0 + n_rec > min(NG, args.ngcap)) {
+        if (pair >= sp.pairs || g0 + n_rec > min(ps.NG, args.ngcap)) {
           atomicOr(args.status, kStatusBounds);
           return;
         }
@@ -822,8 +840,8 @@ decode_kernel(DecodeArgs args, Split sp) {
         bulk_load(dst, args.records + ((long)pair * args.ngcap + g0) * rec_stride, bytes, &bars[k]);
       }
     } else {
-      const int t0 = NG * kGroup + kResTok * (kk - sp.n2 - sp.n1);
-      const int n = min(kResTok, S - t0);
+      const int t0 = ps.NG * kGroup + kResTok * (kk - ps.n2 - ps.n1);
+      const int n = min(kResTok, ps.S - t0);
       const long row0 = (long)pair * kRingSlots + t0 % kRingSlots;
 #ifdef KIVI_DEBUG_BOUNDS
       if (pair >= sp.pairs || n < 1 || t0 % kRingSlots + n > kRingSlots) {
@@ -916,7 +934,7 @@ decode_kernel(DecodeArgs args, Split sp) {
         const float m = __ldcg(pp + h), l = __ldcg(pp + HPK + h);
         const float Mn = fmaxf(Mh[h], m);
         fo[h] = Mh[h] == -INFINITY ? 0.f : exp2f(Mh[h] - Mn);
-        fn[h] = exp2f(m - Mn);
+        fn[h] = m == -INFINITY ? 0.f : exp2f(m - Mn);  // a partial without tokens
         Lh[h] = Lh[h] * fo[h] + l * fn[h];
         Mh[h] = Mn;
       }
@@ -946,7 +964,8 @@ decode_kernel(DecodeArgs args, Split sp) {
       float M = m;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-      const float f = member ? exp2f(m - M) : 0.f;
+      // (a segment may hold only empty items of a short sequence: m = M = -inf)
+      const float f = member && m != -INFINITY ? exp2f(m - M) : 0.f;
       float L = member ? f * st[HPK + h] : 0.f;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
@@ -1109,6 +1128,7 @@ decode_kernel(DecodeArgs args, Split sp) {
   };
 
   int cur_pair = -1;
+  PairShape cur{};
   bool timed_out = false;
   int i_stop = 0;
 
@@ -1126,6 +1146,7 @@ decode_kernel(DecodeArgs args, Split sp) {
       // waits for the item, so that the two latencies overlap
       w.load_pair(args.q + ((long)(pair / args.Hkv) * args.Hq + (long)(pair % args.Hkv) * HPK) * D);
       cur_pair = pair;
+      cur = pair_shape(pair);
     }
     // the next item, claimed now: the counter's latency hides under the item
     const int next = claim();
@@ -1136,12 +1157,12 @@ decode_kernel(DecodeArgs args, Split sp) {
       break;
     }
     unsigned char* base = wbase + k * C::kItemBytes;
-    if (kk < sp.n2 + sp.n1) {
-      w.groups(base, kk < sp.n2);
-    } else {
-      const int t0 = NG * kGroup + kResTok * (kk - sp.n2 - sp.n1);
-      w.residual(base, min(kResTok, S - t0));
-    }
+    if (kk < cur.n2 + cur.n1) {
+      w.groups(base, kk < cur.n2);
+    } else if (kk < cur.n2 + cur.n1 + cur.nr) {
+      const int t0 = cur.NG * kGroup + kResTok * (kk - cur.n2 - cur.n1);
+      w.residual(base, min(kResTok, cur.S - t0));
+    }  // else: an empty item of a shorter sequence
     // release the item slot and start the next item's copies into it (the only
     // generic writes to a slot, residual rows zeroed, are fenced where they happen)
     __syncwarp();
@@ -1284,6 +1305,11 @@ int pair_slots(int D, int bits, int hpk) {
 }
 
 }  // namespace
+
+int decode_items(int S) {
+  const int NG = num_groups(S);
+  return NG / 2 + NG % 2 + (S - NG * kGroup + kResTok - 1) / kResTok;
+}
 
 cudaError_t debug_overstate_copies(unsigned bytes) {
 #ifdef KIVI_DEBUG_BUILD

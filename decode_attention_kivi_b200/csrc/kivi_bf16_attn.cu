@@ -18,14 +18,13 @@
 // written to the output directly, a pair shared with other CTAs as a partial,
 // and the last CTA to arrive at a pair (a ticket per pair) merges its partials.
 // Every wait is bounded; a wait that runs out sets the status word.
-#include <cuda.h>
 #include <cuda_bf16.h>
-#include <cudaTypedefs.h>
 
 #include "kivi_kernels.h"
 #include "kivi_launch.cuh"
 #include "kivi_layout.cuh"
 #include "kivi_ptx.cuh"
+#include "kivi_tmap.cuh"
 
 namespace kivi {
 namespace {
@@ -451,32 +450,6 @@ BSplit make_bsplit(int pairs, int S, int Smax, int num_sms) {
   return s;
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q{};
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
-            cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      p = nullptr;
-    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }();
-  return fn;
-}
-
-// [rows][D] bf16, boxes of 64 channels x 64 rows, 128-byte swizzle.
-bool encode_cache_map(CUtensorMap* map, const void* base, long rows, int D) {
-  const auto fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)kBoxCols, (cuuint32_t)kTile};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int D, int HPK>
 cudaError_t launch_bf16_t(const Bf16DecodeArgs& x, cudaStream_t stream) {
   using C = BCfg<D, HPK>;
@@ -489,7 +462,7 @@ cudaError_t launch_bf16_t(const Bf16DecodeArgs& x, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   const long rows = (long)x.B * x.Hkv * x.Smax;
   CUtensorMap tk, tv;
-  if (!encode_cache_map(&tk, x.k, rows, D) || !encode_cache_map(&tv, x.v, rows, D))
+  if (!encode_bf16_map(&tk, x.k, rows, D, kTile) || !encode_bf16_map(&tv, x.v, rows, D, kTile))
     return cudaErrorInvalidValue;
   const BSplit sp = make_bsplit(x.B * x.Hkv, x.S, x.Smax, x.num_sms);
   Bf16Args a{};

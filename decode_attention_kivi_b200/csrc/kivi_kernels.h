@@ -9,9 +9,10 @@
 namespace kivi {
 
 struct PrefillArgs {
-  const __nv_bfloat16* k;  // [B][Hkv][S][D]
+  const __nv_bfloat16* k;  // [B][Hkv][S][D] (S: the row stride, the longest sequence)
   const __nv_bfloat16* v;
-  int B, Hkv, S, ng, ngcap;
+  const int* lens;         // device [B] tokens per sequence, or null: S for every sequence
+  int B, Hkv, S, ng, ngcap;  // ng = NG(S)
   uint8_t* records;        // layer base [B][Hkv][ngcap] records
   __nv_bfloat16* ring_k;   // layer base [B][Hkv][R+G][D]
   __nv_bfloat16* ring_v;
@@ -20,8 +21,9 @@ struct PrefillArgs {
 struct AppendArgs {
   const __nv_bfloat16* k_new;  // [B][Hkv][D]
   const __nv_bfloat16* v_new;
+  const int* lens;             // device [B] prompt lengths, or null: S for every sequence
+  int steps;                   // appends since the prompt (with lens): S_b = lens[b] + steps
   int B, Hkv, S, ngcap;
-  int flush, ng;               // flush ring tokens [ng*G, ng*G+G) into record ng
   __nv_bfloat16* ring_k;
   __nv_bfloat16* ring_v;
   uint8_t* records;
@@ -37,7 +39,10 @@ struct DecodeArgs {
   int* tickets;                  // one per (sequence, kv head); zero between calls
   float* partials;               // [max_ctas][2][Hq/Hkv][D + 2] split partials
   int max_ctas;                  // capacity of `partials` in CTAs
-  int B, Hkv, Hq, S, ngcap;
+  const int* lens;               // device [B] prompt lengths, or null: S for every sequence
+  int steps;                     // appends since the prompt: S_b = lens[b] + steps
+  int B, Hkv, Hq, S, ngcap;      // S: every sequence's length, or with lens the length
+                                 // whose decode_items the split gives each pair
   float sm_scale;                // <= 0: 1/sqrt(D)
   int num_sms;
   int device;                    // the CUDA device the buffers live on (current at launch)
@@ -81,8 +86,34 @@ cudaError_t launch_bf16_decode(const Bf16DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_fake_quant_keys(int D, int bits, const __nv_bfloat16* k, long rows,
                                    float* k_hat, int per_token, cudaStream_t stream);
 
+// Causal prefill attention on the tcgen05 tensor cores; with `records` set, the
+// CTAs of the first query head of every kv head also quantize their diagonal
+// key/value tile into the cache (groups below NG(S)) and its ring (the rest).
+struct PrefillAttnArgs {
+  const __nv_bfloat16* q;        // [B][Hq][S][D]
+  const __nv_bfloat16* k;        // [B][Hkv][S][D]
+  const __nv_bfloat16* v;        // [B][Hkv][S][D]
+  float* out;                    // [B][Hq][S][D]
+  uint32_t* status;              // device status word, or null
+  int B, Hkv, Hq, S;
+  float sm_scale;                // <= 0: 1/sqrt(D)
+  uint8_t* records;              // this layer's records, or null: attention only
+  __nv_bfloat16* ring_k;         // this layer's rings [B][Hkv][R+G][D]
+  __nv_bfloat16* ring_v;
+  int ngcap;
+  int device;
+};
+
+cudaError_t launch_prefill_attention(int D, int bits, const PrefillAttnArgs& a,
+                                     cudaStream_t stream);
+
 cudaError_t launch_prefill(int D, int bits, const PrefillArgs& a, cudaStream_t stream);
 cudaError_t launch_append(int D, int bits, const AppendArgs& a, cudaStream_t stream);
 cudaError_t launch_decode(int D, int bits, const DecodeArgs& a, cudaStream_t stream);
+
+// Work items the decode split gives one (sequence, kv head) pair of S tokens:
+// record pairs, a lone record, and residual rows of 8 tokens.  Not monotonic in
+// S: just before a flush the residual holds R + G - 1 tokens.
+int decode_items(int S);
 
 }  // namespace kivi

@@ -170,6 +170,59 @@ kivi_status kivi_quantize_prefill(kivi_cache* cache, int32_t layer,
                                   const void* k, const void* v, int32_t S,
                                   void* stream);
 
+/* Prefill with a prompt length per sequence (a ragged batch, as in the serving
+ * setting of the [Llama-3 rec] "Methodology", which batches prompts of
+ * different lengths).  k, v: bf16 [batch][num_kv_heads][S_max][head_dim] on the device;
+ * sequence b uses its first lengths[b] tokens (0 <= lengths[b] <= S_max <=
+ * max_tokens), quantized in groups aligned to its own token 0, the rest of its
+ * residual in its ring.  lengths: host array [batch], read before the call
+ * returns (the call synchronises `stream` once to place them in the workspace).
+ * Every later kivi_append_token adds one token to every sequence (each flushes
+ * on its own schedule), and kivi_decode_attention attends each sequence's own
+ * tokens; kivi_cache_length reports the longest sequence.  The layer must be
+ * empty.  Errors: INVALID_ARG, STATE, CAPACITY (S_max > max_tokens), CUDA. */
+kivi_status kivi_quantize_prefill_ragged(kivi_cache* cache, int32_t layer, const void* k,
+                                         const void* v, int32_t S_max,
+                                         const int32_t* lengths, void* stream);
+
+/* Causal prefill attention with the prompt quantized into `layer` in its
+ * epilogue: the step before decoding ([Llama-3 rec] "KV bytes basis": the
+ * prompt's history is kept as quantized groups, its newest tokens in bf16).
+ * For query head h of sequence b (kv head h / (num_q_heads / num_kv_heads))
+ * and prompt position i,
+ *   out[b][h][i] = sum_{j<=i} softmax_j(sm_scale * <q[b][h][i], k[b][kvh][j]>) v[b][kvh][j],
+ * computed on the tensor cores with bf16 operands, fp32 scores and accumulation,
+ * and the softmax weights rounded to bf16 for the second product.  The layer
+ * then holds exactly what kivi_quantize_prefill(k, v, S) writes (records of the
+ * NG(S) groups, tokens [NG*G, S) in the rings).
+ *   q: bf16 [batch][num_q_heads][S][head_dim]; k, v: bf16 [batch][num_kv_heads]
+ *      [S][head_dim]; out: fp32 [batch][num_q_heads][S][head_dim], written.  All
+ *      device, 16-byte aligned, owned by the caller.
+ *   sm_scale <= 0 means 1/sqrt(head_dim).  S >= 1.
+ * A wait that runs out sets the cache's device status word
+ * (kivi_check_device_status).  Asynchronous on `stream`.
+ * Errors: INVALID_ARG (NULL or unaligned pointers, S < 1, batch * num_q_heads *
+ * (S + 128) >= 2^31, sm_scale not finite), STATE (layer not empty), CAPACITY
+ * (S > max_tokens), CUDA. */
+kivi_status kivi_prefill_attention(kivi_cache* cache, int32_t layer, const void* q,
+                                   const void* k, const void* v, int32_t S, float* out,
+                                   float sm_scale, void* stream);
+
+/* The same causal attention without a cache (for comparisons and for models
+ * that quantize elsewhere).  Arguments as in kivi_prefill_attention, with the
+ * shape given explicitly; head_dim 64 or 128, num_q_heads a multiple of
+ * num_kv_heads.  status: NULL, or a zeroed device uint32 (4-byte aligned) that
+ * a wait that ran out sets to a non-zero code.
+ * Errors: INVALID_ARG, UNSUPPORTED (head_dim, head ratio), CUDA. */
+kivi_status kivi_causal_attention(const void* q, const void* k, const void* v, int32_t batch,
+                                  int32_t num_kv_heads, int32_t num_q_heads, int32_t head_dim,
+                                  int32_t S, float* out, float sm_scale, uint32_t* status,
+                                  void* stream);
+
+/* Token count of every sequence of `layer` (host array S_out[batch]): the
+ * ragged lengths, or the layer's common length.  Errors: INVALID_ARG. */
+kivi_status kivi_cache_lengths(const kivi_cache* cache, int32_t layer, int32_t* S_out);
+
 /* Appends one generated token per sequence to `layer` ([HF page]: the cache
  * grows with every generated token).  k_new, v_new: device bf16 [B][Hkv][D],
  * written to ring slot S mod (R+G).  When S + 1 - NG*G == R + G the same launch

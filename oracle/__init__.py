@@ -18,6 +18,7 @@ from .oracle import (  # noqa: F401
     fake_quant_keys,
     f32_to_f16_bits,
     make_record,
+    prefill_attention,
     num_groups,
     quantize_group,
     record_bytes,

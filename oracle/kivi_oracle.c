@@ -497,3 +497,37 @@ void oracle_fake_quant_keys(const uint16_t* k, int T, int D, int bits, int per_t
     for (int i = 0; i < G; ++i) k_hat[first + i * step] = sh * codes[i] + mh;
   }
 }
+
+/* ------------------------------------------------------------------------ */
+/* Prefill attention over the prompt (causal), the step before the cache     */
+/* ------------------------------------------------------------------------ */
+
+/* Causal attention of a prompt over its own bf16 keys and values, the step whose
+ * epilogue quantizes the prompt into the cache ([Llama-3 rec] "KV bytes basis":
+ * the history is quantized, the newest tokens stay in full precision).  For
+ * query head h of sequence b (kv head h / (Hq / Hkv)) and position i:
+ *   out[b][h][i] = sum_{j <= i} softmax_j(sm_scale * <q_i, k_j>) v_j,  in double.
+ * q: bf16 bits [B][Hq][S][D]; k, v: [B][Hkv][S][D]; out: [B][Hq][S][D]. */
+void oracle_prefill_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B,
+                              int Hkv, int Hq, int S, int D, double sm_scale, double* out) {
+  const int per_kv = Hq / Hkv;
+  double* K = (double*)malloc(sizeof(double) * (size_t)(S > 0 ? S : 1) * D);
+  double* V = (double*)malloc(sizeof(double) * (size_t)(S > 0 ? S : 1) * D);
+  for (int b = 0; b < B; ++b) {
+    for (int kvh = 0; kvh < Hkv; ++kvh) {
+      const long base = ((long)b * Hkv + kvh) * S * D;
+      for (long i = 0; i < (long)S * D; ++i) {
+        K[i] = bf16_bits_to_float(k[base + i]);
+        V[i] = bf16_bits_to_float(v[base + i]);
+      }
+      for (int j = 0; j < per_kv; ++j) {
+        const long head = (long)b * Hq + (long)kvh * per_kv + j;
+        for (int i = 0; i < S; ++i)  /* position i sees tokens 0..i */
+          attend_dense(K, V, q + (head * S + i) * D, i + 1, D, sm_scale,
+                       out + (head * S + i) * D);
+      }
+    }
+  }
+  free(K);
+  free(V);
+}

@@ -80,6 +80,8 @@ def _c():
         lib.oracle_attention.restype = None
         lib.oracle_attention_bf16.argtypes = [u16p, u16p, u16p, i, i, i, i, i, i, d, f64p]
         lib.oracle_attention_bf16.restype = None
+        lib.oracle_prefill_attention.argtypes = [u16p, u16p, u16p, i, i, i, i, i, d, f64p]
+        lib.oracle_prefill_attention.restype = None
         lib.oracle_fake_quant_keys.argtypes = [u16p, i, i, i, i, f64p]
         lib.oracle_fake_quant_keys.restype = None
         _lib = lib
@@ -178,6 +180,24 @@ def attention_bf16(k: np.ndarray, v: np.ndarray, q: np.ndarray, S: int | None = 
     _c().oracle_attention_bf16(_p(k, ctypes.c_uint16), _p(v, ctypes.c_uint16),
                                _p(q, ctypes.c_uint16), B, Hkv, Hq, S, Smax, D, scale,
                                _p(out, ctypes.c_double))
+    return out
+
+
+def prefill_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray,
+                      sm_scale: float | None = None) -> np.ndarray:
+    """Causal attention of a prompt: q bf16 bits [B][Hq][S][D], k, v [B][Hkv][S][D]
+    -> float64 [B][Hq][S][D]; position i attends tokens 0..i."""
+    q = np.ascontiguousarray(q, np.uint16)
+    k = np.ascontiguousarray(k, np.uint16)
+    v = np.ascontiguousarray(v, np.uint16)
+    B, Hq, S, D = q.shape
+    Hkv = k.shape[1]
+    assert k.shape == (B, Hkv, S, D) and v.shape == k.shape and Hq % Hkv == 0
+    scale = 1.0 / math.sqrt(D) if sm_scale is None or sm_scale <= 0 else float(sm_scale)
+    out = np.zeros((B, Hq, S, D), np.float64)
+    _c().oracle_prefill_attention(_p(q, ctypes.c_uint16), _p(k, ctypes.c_uint16),
+                                  _p(v, ctypes.c_uint16), B, Hkv, Hq, S, D, scale,
+                                  _p(out, ctypes.c_double))
     return out
 
 

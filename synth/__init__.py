@@ -57,7 +57,7 @@ WORKLOADS = {
 }
 
 # Tensor tags mixed into the per-tensor seed.
-_TAG_KEY_SCALE, _TAG_K, _TAG_V, _TAG_Q, _TAG_KNEW, _TAG_VNEW = 1, 2, 3, 4, 5, 6
+_TAG_KEY_SCALE, _TAG_K, _TAG_V, _TAG_Q, _TAG_KNEW, _TAG_VNEW, _TAG_QPROMPT = 1, 2, 3, 4, 5, 6, 7
 
 
 def _gen(w: Workload, tag: int, layer: int, step: int, device) -> torch.Generator:
@@ -111,6 +111,14 @@ def query(w: Workload, layer: int, step: int, device="cpu"):
     """Decode query of step `step`, bf16 [B][Hq][D]."""
     shape = (w.batch, w.num_q_heads, w.head_dim)
     q = torch.randn(shape, generator=_gen(w, _TAG_Q, layer, step, device), device=device)
+    return q.to(torch.bfloat16)
+
+
+def prompt_query(w: Workload, layer: int, S: int | None = None, device="cpu"):
+    """Queries of the prompt's positions (prefill attention), bf16 [B][Hq][S][D]."""
+    S = w.context if S is None else S
+    shape = (w.batch, w.num_q_heads, S, w.head_dim)
+    q = torch.randn(shape, generator=_gen(w, _TAG_QPROMPT, layer, 0, device), device=device)
     return q.to(torch.bfloat16)
 
 

@@ -61,7 +61,9 @@ def test_required_bytes_layout(lib):
     # (m, l, acc) partials of the 4 query heads of a kv head per CTA, for 256 CTAs
     pairs = 16 * 8
     tickets = (4 * pairs + 255) // 256 * 256
-    assert s.workspace_bytes == 256 + tickets + 256 * 2 * 4 * (128 + 2) * 4
+    # then the prompt lengths of ragged layers, [32 layers][16 sequences] int32
+    lens = (32 * 16 * 4 + 255) // 256 * 256
+    assert s.workspace_bytes == 256 + tickets + 256 * 2 * 4 * (128 + 2) * 4 + lens
 
 
 @pytest.mark.parametrize("field,value,code", [
@@ -174,3 +176,28 @@ def test_record_layout_query(lib):
         assert rb.value == O2.record_bytes(D, bits)
         assert ng.value == O2.num_groups(mt)
     assert N.STATUS[lib.kivi_record_layout(None, None, None)] == "KIVI_ERR_INVALID_ARG"
+
+
+def test_ragged_entry_points_validate_without_a_handle(lib):
+    lens = (ctypes.c_int32 * 2)(3, 5)
+    assert N.STATUS[lib.kivi_quantize_prefill_ragged(None, 0, None, None, 8, lens, None)] == \
+        "KIVI_ERR_INVALID_ARG"
+    out = (ctypes.c_int32 * 2)()
+    assert N.STATUS[lib.kivi_cache_lengths(None, 0, out)] == "KIVI_ERR_INVALID_ARG"
+
+
+def test_prefill_attention_validation(lib):
+    """Host checks of the prefill-attention entry points (no launch on these paths)."""
+    fake = 1 << 20
+    call = lambda B, hkv, hq, D, S, q=fake, status=None: lib.kivi_causal_attention(  # noqa: E731
+        q, fake, fake, B, hkv, hq, D, S, fake, 0.0, status, None)
+    assert N.STATUS[call(1, 8, 32, 128, 0)] == "KIVI_ERR_INVALID_ARG"        # S < 1
+    assert N.STATUS[call(0, 8, 32, 128, 10)] == "KIVI_ERR_INVALID_ARG"       # no sequences
+    assert N.STATUS[call(1, 8, 20, 128, 10)] == "KIVI_ERR_UNSUPPORTED"       # Hq % Hkv
+    assert N.STATUS[call(1, 8, 32, 96, 10)] == "KIVI_ERR_UNSUPPORTED"        # head_dim
+    assert N.STATUS[call(1, 8, 32, 128, 10, q=fake + 2)] == "KIVI_ERR_INVALID_ARG"   # unaligned
+    assert N.STATUS[call(1, 8, 32, 128, 10, q=None)] == "KIVI_ERR_INVALID_ARG"       # NULL
+    assert N.STATUS[call(1, 8, 32, 128, 10, status=fake + 2)] == "KIVI_ERR_INVALID_ARG"
+    assert N.STATUS[call(4096, 8, 32, 128, 1 << 14)] == "KIVI_ERR_INVALID_ARG"  # rows >= 2^31
+    assert N.STATUS[lib.kivi_prefill_attention(None, 0, fake, fake, fake, 16, fake, 0.0,
+                                               None)] == "KIVI_ERR_INVALID_ARG"

@@ -502,3 +502,23 @@ def test_fake_quant_keys_exact_on_its_own_grid(bits):
     assert np.array_equal(O.fake_quant_keys(_bits(kt), bits, True), kt.numpy())
     # and the other granularity is not exact on them
     assert not np.array_equal(O.fake_quant_keys(_bits(kc), bits, True), kc.numpy())
+
+
+# ---------------------------------------------------------------------------
+# Prefill attention (causal), the step before the cache is filled
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("B,Hkv,Hq,S,D", [(1, 1, 1, 1, 64), (2, 2, 8, 70, 64), (1, 2, 2, 33, 128)])
+def test_prefill_attention_equals_causal_sdpa(B, Hkv, Hq, S, D):
+    rng = np.random.default_rng(S + Hq)
+    q = torch.tensor(rng.standard_normal((B, Hq, S, D))).to(torch.bfloat16)
+    k = torch.tensor(rng.standard_normal((B, Hkv, S, D))).to(torch.bfloat16)
+    v = torch.tensor(rng.standard_normal((B, Hkv, S, D))).to(torch.bfloat16)
+    out = O.prefill_attention(_bits(q), _bits(k), _bits(v))
+    rep = Hq // Hkv
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q.double(), k.double().repeat_interleave(rep, 1), v.double().repeat_interleave(rep, 1),
+        is_causal=True, scale=1 / math.sqrt(D)).numpy()
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+    # position 0 sees only token 0: its value row, exactly
+    np.testing.assert_array_equal(out[:, :, 0], v.double().numpy().repeat(rep, 1)[:, :, 0])

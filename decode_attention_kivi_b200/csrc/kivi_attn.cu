@@ -717,7 +717,9 @@ struct Warp {
   }
 };
 
-template <int D, int BITS, int HPK>
+// RAGGED: a length per sequence (args.lens); otherwise every pair has the split's
+// shape and the per-pair checks compile away.
+template <int D, int BITS, int HPK, bool RAGGED>
 __global__ void __launch_bounds__(Cfg<D, BITS, HPK>::kThreads, 1)
 decode_kernel(DecodeArgs args, Split sp) {
   using C = Cfg<D, BITS, HPK>;
@@ -794,7 +796,7 @@ decode_kernel(DecodeArgs args, Split sp) {
   // items of a shorter one past its own count are empty)
   struct PairShape { int S, NG, n2, n1, nr; };
   auto pair_shape = [&](int pair) -> PairShape {
-    if (args.lens == nullptr) return PairShape{args.S, sp.NG, sp.n2, sp.n1, sp.nr};
+    if constexpr (!RAGGED) return PairShape{args.S, sp.NG, sp.n2, sp.n1, sp.nr};
     PairShape p;
     p.S = __ldg(args.lens + pair / args.Hkv) + args.steps;
     p.NG = num_groups(p.S);
@@ -821,7 +823,7 @@ decode_kernel(DecodeArgs args, Split sp) {
     unsigned char* dst = wbase + k * C::kItemBytes;
     const int pair = pair_of(sp, it), kk = it - pair * sp.ipp;
     const PairShape ps = pair_shape(pair);
-    if (kk >= ps.n2 + ps.n1 + ps.nr) {  // past this sequence's items: nothing to copy
+    if (RAGGED && kk >= ps.n2 + ps.n1 + ps.nr) {  // past this sequence's items: nothing to copy
       if (lane == 0) mbar_arrive(&bars[k]);
       return;
     }
@@ -1159,7 +1161,7 @@ decode_kernel(DecodeArgs args, Split sp) {
     unsigned char* base = wbase + k * C::kItemBytes;
     if (kk < cur.n2 + cur.n1) {
       w.groups(base, kk < cur.n2);
-    } else if (kk < cur.n2 + cur.n1 + cur.nr) {
+    } else if (!RAGGED || kk < cur.n2 + cur.n1 + cur.nr) {
       const int t0 = cur.NG * kGroup + kResTok * (kk - cur.n2 - cur.n1);
       w.residual(base, min(kResTok, cur.S - t0));
     }  // else: an empty item of a shorter sequence
@@ -1239,16 +1241,16 @@ Split make_split(int pairs, int S, int num_sms) {
   return s;
 }
 
-template <int D, int BITS, int HPK>
-cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t stream) {
+template <int D, int BITS, int HPK, bool RAGGED>
+cudaError_t launch_decode_r(const DecodeArgs& a, cudaStream_t stream) {
   using C = Cfg<D, BITS, HPK>;
   int unused = 0;
   cudaError_t e = per_device_setup(a.device, &unused, [](int* v) {
     *v = 1;
-    cudaError_t r = cudaFuncSetAttribute(decode_kernel<D, BITS, HPK>,
+    cudaError_t r = cudaFuncSetAttribute(decode_kernel<D, BITS, HPK, RAGGED>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::kBytes);
     if (r != cudaSuccess) return r;
-    return cudaFuncSetAttribute(decode_kernel<D, BITS, HPK>,
+    return cudaFuncSetAttribute(decode_kernel<D, BITS, HPK, RAGGED>,
                                 cudaFuncAttributePreferredSharedMemoryCarveout,
                                 (int)cudaSharedmemCarveoutMaxShared);
   });
@@ -1257,10 +1259,16 @@ cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t stream) {
   if (pairs > (1L << 30) / 4096) return cudaErrorInvalidValue;  // keeps the cost axis in int
   const Split sp = make_split<D, BITS, HPK>((int)pairs, a.S, a.num_sms);
   if ((long)sp.pairs * sp.pc >= (1L << 31) || sp.n > a.max_ctas) return cudaErrorInvalidValue;
-  e = launch_pdl(decode_kernel<D, BITS, HPK>, dim3(sp.n), dim3(C::kThreads), C::kBytes, stream,
-                 a, sp);
+  e = launch_pdl(decode_kernel<D, BITS, HPK, RAGGED>, dim3(sp.n), dim3(C::kThreads), C::kBytes,
+                 stream, a, sp);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+template <int D, int BITS, int HPK>
+cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t stream) {
+  return a.lens != nullptr ? launch_decode_r<D, BITS, HPK, true>(a, stream)
+                           : launch_decode_r<D, BITS, HPK, false>(a, stream);
 }
 
 template <int D, int BITS>

@@ -12,25 +12,35 @@
 //   out[b][h][i] = sum_{j <= i} softmax_j(sm_scale * <q_i, k_j>) v_j.
 //
 // One CTA per (query tile of 128 positions, sequence, query head), the tiles
-// with the most key tiles first.  Six warps:
-//   warp 4 (producer)  2D tensor copies of Q once and of K and V tiles of 128
-//                      keys into a two-stage ring (128-byte swizzle);
-//   warp 5 (MMA)       one thread issues S_j = Q K_j^T (M = N = 128, K = D) into
+// with the most key tiles first.  Twelve warps:
+//   warp 8 (producer)  2D tensor copies of Q once and of K and V tiles of 128
+//                      keys into two-stage rings (128-byte swizzle), the
+//                      diagonal tile first, then towards key 0; a K stage is
+//                      refilled once its scores are computed, a V stage once
+//                      its product is;
+//   warp 9 (MMA)       one thread issues S_j = Q K_j^T (M = N = 128, K = D) into
 //                      one of two TMEM score buffers, and O += P_j V_j (M = 128,
 //                      N = D, K = 128) into the TMEM output, each followed by a
 //                      commit to an mbarrier;
-//   warps 0-3          one query row per thread (its TMEM lane): the row of S_j
-//                      from TMEM, the causal mask on the diagonal tile, the
-//                      online softmax in base 2, P_j as bf16 into shared memory
-//                      in the operand layout of the second MMA.  The output is
-//                      rescaled in TMEM only when a row maximum grew by more
-//                      than 2^8 (up to then the stale maximum is kept: the
-//                      weights stay below 2^8 and O / l is unchanged).
-// S_{j+1} is computed while the softmax works on S_j.  With the quantize on,
-// the CTAs of the first query head of each kv head turn their diagonal K and V
-// tile (still in shared memory after the last MMA) into group records (groups
-// below NG(S)) and ring rows (tokens NG(S)*G .. S-1) with the quantizer of the
-// quantize kernels, bit for bit.
+//   warps 0-7          half a query row per thread (warps w and w + 4 share the
+//                      TMEM lanes of rows 32 (w mod 4) + lane and take 64 keys
+//                      each): the row of S_j from TMEM, the causal mask on the
+//                      diagonal tile, the online softmax in base 2 (the halves
+//                      exchange their maxima once per tile) with the weights
+//                      computed while the tensor cores finish P_{j-1} V_{j-1},
+//                      then P_j as bf16 into shared memory in the operand layout
+//                      of the second MMA.  The output is rescaled in TMEM only
+//                      when a row maximum grew by more than 2^8 (up to then the
+//                      stale maximum is kept: the weights stay below 2^8 and
+//                      O / l is unchanged);
+//   warps 10-11        with the quantize on, in the CTAs of the longer half of
+//                      the query tiles: this CTA's share of the groups of key
+//                      tiles qt and nqt - 1 - qt (query head j < 4 of a kv head
+//                      takes groups j, j + min(HPK, 4), ...): group records
+//                      below NG(S), ring rows for tokens NG(S)*G .. S-1, with the
+//                      quantizer of the quantize kernels, bit for bit, while the
+//                      other warps run the attention.
+// S_{j+1} is computed while the softmax works on S_j.
 //
 // TMEM: 512 columns (one CTA per SM): scores at columns 0 and 128, O at 256.
 // Every mbarrier wait is bounded; a wait that runs out sets the status word,
@@ -52,16 +62,20 @@ namespace {
 
 constexpr int kTileM = 128;                   // query rows per CTA = TMEM lanes
 constexpr int kTileN = 128;                   // keys per tile
-constexpr int kSoftWarps = 4;
+constexpr int kSoftWarps = 8;                 // two per TMEM lane quarter: each row is split
+                                              // into two halves of 64 keys
+constexpr int kHalfN = kTileN / 2;
 constexpr int kProducerWarp = kSoftWarps;
 constexpr int kMmaWarp = kSoftWarps + 1;
-constexpr int kThreadsPA = (kSoftWarps + 2) * 32;
+constexpr int kQuantWarp0 = kSoftWarps + 2;   // two warps that quantize the prompt
+constexpr int kQuantThreadsPA = 64;
+constexpr int kThreadsPA = (kSoftWarps + 2) * 32 + kQuantThreadsPA;
 constexpr int kSlabBytes = 128 * 128;         // 64 bf16 columns of 128 rows
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kStatusWaitTimeoutPA = 1u;
 constexpr float kLog2ePA = 1.4426950408889634f;
 constexpr float kRescaleSlack = 8.f;          // log2 growth of a row max before O is rescaled
-constexpr int kSoftBarrier = 1;               // named barrier of the softmax warps
+constexpr int kQuantBarrier = 1;              // named barrier of the quantize warps
 
 template <int D>
 struct PACfg {
@@ -70,18 +84,22 @@ struct PACfg {
   static constexpr int kOffQ = 0;
   static constexpr int kOffKV = kOffQ + kTileBytes;       // stage s: K at 2s, V at 2s + 1
   static constexpr int kOffP = kOffKV + 4 * kTileBytes;
-  static constexpr int kOffBars = kOffP + 2 * kSlabBytes; // P: 128 rows x 128 keys
+  static constexpr int kOffQuant = kOffP + 2 * kSlabBytes; // P: 128 rows x 128 keys
+  static constexpr int kOffMax = kOffQuant + (int)sizeof(quant::QuantSmem<D>);  // [2][2][128] f32
+  static constexpr int kOffBars = kOffMax + 2 * 2 * kTileM * 4;
   static constexpr int kUsed = kOffBars + 256;
   // more than half of the SM's shared memory: one CTA per SM, which holds all
   // 512 TMEM columns
   static constexpr int kBytes = kUsed + 1024 > 120 * 1024 ? kUsed + 1024 : 120 * 1024;
   static constexpr uint32_t kColS = 0, kColO = 2 * kTileN;
   static_assert(kColO + D <= kTmemCols, "TMEM plan");
-  static_assert(sizeof(quant::QuantSmem<D>) <= 2 * kSlabBytes, "quantize tiles fit in P");
+  static_assert(sizeof(quant::QuantSmem<D>) % 16 == 0, "barriers stay aligned");
   static_assert(kBytes <= 227 * 1024, "shared-memory plan");
 };
 
 struct PAParams {
+  const __nv_bfloat16* k;  // the prompt's keys and values, read by the quantize warps
+  const __nv_bfloat16* v;
   float* out;
   uint32_t* status;
   int B, Hkv, Hq, S, nqt, NG, ngcap;
@@ -110,16 +128,20 @@ prefill_attention_kernel(const __grid_constant__ CUtensorMap tq,
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // K and V stages have their own barriers: a K stage is free once its scores
+  // are computed, long before the V stage of the same tile.
   uint64_t* q_full = reinterpret_cast<uint64_t*>(smem + C::kOffBars);
-  uint64_t* kv_full = q_full + 1;   // [2]
-  uint64_t* kv_empty = q_full + 3;  // [2]
-  uint64_t* s_full = q_full + 5;    // [2]
-  uint64_t* p_full = q_full + 7;
-  uint64_t* o_done = q_full + 8;
-  uint64_t* drained = q_full + 9;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(q_full + 10);
+  uint64_t* k_full = q_full + 1;    // [2]
+  uint64_t* k_empty = q_full + 3;   // [2]
+  uint64_t* v_full = q_full + 5;    // [2]
+  uint64_t* v_empty = q_full + 7;   // [2]
+  uint64_t* s_full = q_full + 9;    // [2]
+  uint64_t* p_full = q_full + 11;
+  uint64_t* o_done = q_full + 12;
+  uint64_t* drained = q_full + 13;
+  uint64_t* half_bar = q_full + 14;  // [4 lane quarters][2 tile parities]: row-max exchange
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(q_full + 22);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
-  volatile int* s_ok = s_abort + 1;  // [kSoftWarps]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int BH = a.B * a.Hq;
@@ -135,13 +157,16 @@ prefill_attention_kernel(const __grid_constant__ CUtensorMap tq,
     *s_abort = 0;
     mbar_init(q_full, 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
     }
     mbar_init(p_full, kSoftWarps * 32);
     mbar_init(o_done, 1);
     mbar_init(drained, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(&half_bar[i], 64);
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -162,27 +187,39 @@ prefill_attention_kernel(const __grid_constant__ CUtensorMap tq,
       mbar_expect_tx(q_full, C::kTileBytes);
       for (int sl = 0; sl < C::kSlabs; ++sl)
         tma_load_2d(smem + C::kOffQ + sl * kSlabBytes, &tq, 64 * sl, q_row0, q_full);
-      int issued = 0;
-      for (int j = 0; j < nt; ++j) {
+      // tile j (the diagonal tile first, then towards key 0) goes to stage j mod 2;
+      // K(j + 1) is issued before V(j): it is needed first and freed first
+      auto issue = [&](int j, bool is_k) -> bool {
         const int st = j & 1;
-        if (j >= 2 && !mbar_wait_bounded(&kv_empty[st], ((j >> 1) - 1) & 1)) {
-          fail();
-          break;
+        uint64_t* empty = is_k ? &k_empty[st] : &v_empty[st];
+        if (j >= 2 && !mbar_wait_bounded(empty, ((j >> 1) - 1) & 1)) return false;
+        if (*s_abort) return false;
+        uint64_t* full = is_k ? &k_full[st] : &v_full[st];
+        unsigned char* dst = smem + C::kOffKV + (2 * st + (is_k ? 0 : 1)) * C::kTileBytes;
+        const int row = kv_row0 + (qt - j) * kTileN;
+        mbar_expect_tx(full, C::kTileBytes);
+        for (int sl = 0; sl < C::kSlabs; ++sl)
+          tma_load_2d(dst + sl * kSlabBytes, is_k ? &tk : &tv, 64 * sl, row, full);
+        return true;
+      };
+      int issued_k = 0, issued_v = 0;
+      bool ok = issue(0, true);
+      if (ok) issued_k = 1;
+      for (int j = 0; ok && j < nt; ++j) {
+        if (j + 1 < nt) {
+          if (!(ok = issue(j + 1, true))) break;
+          issued_k = j + 2;
         }
-        if (*s_abort) break;
-        unsigned char* kdst = smem + C::kOffKV + 2 * st * C::kTileBytes;
-        unsigned char* vdst = kdst + C::kTileBytes;
-        mbar_expect_tx(&kv_full[st], 2 * C::kTileBytes);
-        for (int sl = 0; sl < C::kSlabs; ++sl) {
-          tma_load_2d(kdst + sl * kSlabBytes, &tk, 64 * sl, kv_row0 + j * kTileN, &kv_full[st]);
-          tma_load_2d(vdst + sl * kSlabBytes, &tv, 64 * sl, kv_row0 + j * kTileN, &kv_full[st]);
-        }
-        issued = j + 1;
+        if (!(ok = issue(j, false))) break;
+        issued_v = j + 1;
       }
+      if (!ok) fail();
       // every copy issued lands before the CTA may exit
       if (!mbar_wait_bounded(q_full, 0)) fail();
-      for (int j = issued > 2 ? issued - 2 : 0; j < issued; ++j)
-        if (!mbar_wait_bounded(&kv_full[j & 1], (j >> 1) & 1)) fail();
+      for (int j = issued_k > 2 ? issued_k - 2 : 0; j < issued_k; ++j)
+        if (!mbar_wait_bounded(&k_full[j & 1], (j >> 1) & 1)) fail();
+      for (int j = issued_v > 2 ? issued_v - 2 : 0; j < issued_v; ++j)
+        if (!mbar_wait_bounded(&v_full[j & 1], (j >> 1) & 1)) fail();
     }
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
@@ -200,22 +237,24 @@ prefill_attention_kernel(const __grid_constant__ CUtensorMap tq,
                        tc::desc_sw128(k_base + off, 16, 1024), id_s, s > 0);
         }
         tc::commit(&s_full[st]);
+        tc::commit(&k_empty[st]);
       };
-      bool ok = mbar_wait_bounded(q_full, 0) && mbar_wait_bounded(&kv_full[0], 0);
+      bool ok = mbar_wait_bounded(q_full, 0) && mbar_wait_bounded(&k_full[0], 0);
       if (ok) {
         tc::fence_after();
         issue_scores(0);
       }
       for (int j = 0; ok && j < nt; ++j) {
         if (j + 1 < nt) {
-          if (!mbar_wait_bounded(&kv_full[(j + 1) & 1], ((j + 1) >> 1) & 1)) {
+          if (!mbar_wait_bounded(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1)) {
             ok = false;
             break;
           }
           tc::fence_after();
           issue_scores(j + 1);  // its buffer was read by the softmax of tile j - 1
         }
-        if (!mbar_wait_bounded(p_full, j & 1) || *s_abort) {
+        if (!mbar_wait_bounded(p_full, j & 1) || !mbar_wait_bounded(&v_full[j & 1], (j >> 1) & 1) ||
+            *s_abort) {
           ok = false;
           break;
         }
@@ -229,7 +268,7 @@ prefill_attention_kernel(const __grid_constant__ CUtensorMap tq,
                        tc::desc_sw128(v_base + s * 16 * 128, kSlabBytes, 1024), id_o,
                        j > 0 || s > 0);
         }
-        tc::commit(&kv_empty[j & 1]);
+        tc::commit(&v_empty[j & 1]);
         tc::commit(o_done);
       }
       if (!ok) fail();
@@ -237,17 +276,24 @@ prefill_attention_kernel(const __grid_constant__ CUtensorMap tq,
       tc::commit(drained);
       if (!mbar_wait_bounded(drained, 0)) fail();
     }
-  } else {
-    // Softmax warps: thread r owns query row r of the tile (TMEM lane r).
-    const int r = threadIdx.x;
+  } else if (warp < kSoftWarps) {
+    // Softmax warps: warps w and w + 4 share query rows 32 (w mod 4) + lane (their
+    // TMEM lanes); warp w takes keys [64 h, 64 h + 64) of each tile, h = w / 4.
+    // The two halves of a row exchange their maxima once per tile (through
+    // shared memory and an mbarrier, so a partner that stopped cannot hang it)
+    // and keep separate partial sums, added once at the end.
+    const int quarter = warp & 3, h = warp >> 2;
+    const int r = quarter * 32 + lane;
     const int qpos = qt * kTileM + r;
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     unsigned char* prow = smem + C::kOffP;
+    float* s_max = reinterpret_cast<float*>(smem + C::kOffMax);  // [parity][half][row]
     auto wait_warp = [&](uint64_t* bar, uint32_t parity) {
       const bool w = mbar_wait_bounded(bar, parity);
       return __all_sync(0xffffffffu, w && !*s_abort);
     };
-    float m = -INFINITY, l = 0.f;
+    const float sl2 = a.scale_log2;
+    float m = -INFINITY, l = 0.f;  // running max (log2 units); this half's sum of weights
     bool ok = true;
     for (int j = 0; j < nt; ++j) {
       const int st = j & 1;
@@ -256,26 +302,43 @@ prefill_attention_kernel(const __grid_constant__ CUtensorMap tq,
         break;
       }
       tc::fence_after();
-      float s[kTileN];
-      tc::ld_x128(lane_base + C::kColS + st * kTileN, s);
-      float mx = -INFINITY;
-      if (j == qt) {  // diagonal tile: keys after the query are masked
+      float s[kHalfN];
+      tc::ld_x64(lane_base + C::kColS + st * kTileN + h * kHalfN, s);
+      if (j == 0) {  // the diagonal tile: keys after the query are masked
 #pragma unroll
-        for (int c = 0; c < kTileN; ++c) {
-          s[c] = c <= r ? s[c] * a.scale_log2 : -INFINITY;
-          mx = fmaxf(mx, s[c]);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < kTileN; ++c) {
-          s[c] *= a.scale_log2;
-          mx = fmaxf(mx, s[c]);
-        }
+        for (int c = 0; c < kHalfN; ++c) s[c] = h * kHalfN + c <= r ? s[c] : -INFINITY;
       }
-      const float m_new = fmaxf(m, mx);
+      float mx8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx8[i] = s[i];
+#pragma unroll
+      for (int c = 8; c < kHalfN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      // the other half's maximum (slot parity j: reused two tiles later, after
+      // the partner has passed the next exchange)
+      s_max[(st * 2 + h) * kTileM + r] = mx;
+      mbar_arrive(&half_bar[quarter * 2 + st]);
+      if (!wait_warp(&half_bar[quarter * 2 + st], (j >> 1) & 1)) {
+        ok = false;
+        break;
+      }
+      mx = fmaxf(mx, s_max[(st * 2 + (h ^ 1)) * kTileM + r]);
+      // scores scaled into log2 units inside the exponent's FMA (sl2 > 0 keeps the max)
+      const float m_new = fmaxf(m, mx * sl2);
       const bool grow = m_new > m + kRescaleSlack;  // always at the first tile (m = -inf)
       const float m_use = grow ? m_new : m;
       const float alpha = fast_exp2(m - m_use);     // 1 when kept, 0 at the first tile
+      // the weights of this tile while the tensor cores still work on the last one
+      uint32_t pk[kHalfN / 2];
+      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c = 0; c < kHalfN; c += 2) {
+        const float p0 = fast_exp2(fmaf(s[c], sl2, -m_use));
+        const float p1 = fast_exp2(fmaf(s[c + 1], sl2, -m_use));
+        sum4[(c >> 1) & 3] += p0 + p1;
+        pk[c >> 1] = pack_bf16x2(p0, p1);
+      }
       if (j > 0) {
         // O holds P_{j-1} V_{j-1}, and the P buffer is free again
         if (!wait_warp(o_done, (j - 1) & 1)) {
@@ -285,7 +348,7 @@ prefill_attention_kernel(const __grid_constant__ CUtensorMap tq,
         tc::fence_after();
         if (__any_sync(0xffffffffu, grow)) {  // TMEM loads and stores are warp-wide
 #pragma unroll 1
-          for (int c0 = 0; c0 < D; c0 += 32) {
+          for (int c0 = h * (D / 2); c0 < (h + 1) * (D / 2); c0 += 32) {
             float o[32];
             tc::ld_x32(lane_base + C::kColO + c0, o);
 #pragma unroll
@@ -295,23 +358,11 @@ prefill_attention_kernel(const __grid_constant__ CUtensorMap tq,
           tc::wait_st();
         }
       }
-      float sum = 0.f;
 #pragma unroll
-      for (int c8 = 0; c8 < kTileN / 8; ++c8) {
-        uint4 w;
-        float p[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          p[e] = fast_exp2(s[8 * c8 + e] - m_use);
-          sum += p[e];
-        }
-        w.x = pack_bf16x2(p[0], p[1]);
-        w.y = pack_bf16x2(p[2], p[3]);
-        w.z = pack_bf16x2(p[4], p[5]);
-        w.w = pack_bf16x2(p[6], p[7]);
-        *reinterpret_cast<uint4*>(prow + sw128_offset(r, c8)) = w;
-      }
-      l = l * alpha + sum;
+      for (int c8 = 0; c8 < kHalfN / 8; ++c8)
+        *reinterpret_cast<uint4*>(prow + sw128_offset(r, h * (kHalfN / 8) + c8)) =
+            make_uint4(pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]);
+      l = l * alpha + ((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
       m = m_use;
       fence_proxy_async();  // P is read by the tensor cores
       tc::fence_before();
@@ -319,11 +370,20 @@ prefill_attention_kernel(const __grid_constant__ CUtensorMap tq,
     }
     if (ok) ok = wait_warp(o_done, (nt - 1) & 1);
     if (ok) {
+      // the row's sum: this half's plus the other's (slot parity of tile nt,
+      // whose exchange never happens)
+      const int sp = nt & 1;
+      s_max[(sp * 2 + h) * kTileM + r] = l;
+      mbar_arrive(&half_bar[quarter * 2 + sp]);
+      ok = wait_warp(&half_bar[quarter * 2 + sp], (nt >> 1) & 1);
+      if (ok) l += s_max[(sp * 2 + (h ^ 1)) * kTileM + r];
+    }
+    if (ok) {
       tc::fence_after();
       const float inv = 1.f / l;
       float* orow = a.out + ((long)bh * a.S + qpos) * D;
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
+      for (int c0 = h * (D / 2); c0 < (h + 1) * (D / 2); c0 += 32) {
         float o[32];
         tc::ld_x32(lane_base + C::kColO + c0, o);
         if (qpos < a.S) {
@@ -336,47 +396,49 @@ prefill_attention_kernel(const __grid_constant__ CUtensorMap tq,
     } else {
       fail();
     }
-    if (lane == 0) s_ok[warp] = ok ? 1 : 0;
-    named_sync(kSoftBarrier, kSoftWarps * 32);
-    bool all_ok = true;
-#pragma unroll
-    for (int w = 0; w < kSoftWarps; ++w) all_ok = all_ok && s_ok[w] != 0;
-
-    // Fused quantize of the diagonal tile: every MMA has completed (all four
-    // warps saw the last commit), so the stage of tile qt still holds K_qt and
-    // V_qt and the P buffer is free for the quantizer's tiles.
-    if (all_ok && a.records != nullptr && hq % hpk == 0) {
+  } else {
+    // Quantize warps, running beside the attention: the CTAs of query tile qt
+    // with qt >= nqt - 1 - qt (the longer half) quantize key tile qt and its
+    // partner tile nqt - 1 - qt, so the work hides under their longer attention
+    // and every tile is taken once.  Query head j < 4 of a kv head takes groups
+    // j, j + min(HPK, 4), ... of a tile's four.  Rows are read from global
+    // memory (tile qt right behind the producer's copy; low tiles are read by
+    // every CTA of the kv head and stay in L2).
+    const int hi = hq % hpk, nq = hpk < 4 ? hpk : 4;
+    const int partner = a.nqt - 1 - qt;
+    if (a.records != nullptr && hi < 4 && qt >= partner) {
       constexpr RecordGeom geo{D, BITS};
-      auto& qs = *reinterpret_cast<quant::QuantSmem<D>*>(smem + C::kOffP);
-      const unsigned char* kt = smem + C::kOffKV + 2 * (qt & 1) * C::kTileBytes;
-      const unsigned char* vt = kt + C::kTileBytes;
+      const int qtid = threadIdx.x - kQuantWarp0 * 32;
+      auto& qs = *reinterpret_cast<quant::QuantSmem<D>*>(smem + C::kOffQuant);
       const long seq = (long)b * a.Hkv + kvh;
-      auto sync = [] { named_sync(kSoftBarrier, kSoftWarps * 32); };
-      for (int gi = 0; gi < kTileN / kGroup; ++gi) {
-        const int t0 = qt * kTileN + gi * kGroup;  // the group's first token
-        if (t0 >= a.S) break;
-        const int g = t0 / kGroup;
-        if (g < a.NG) {
-          for (int i = r; i < kGroup * (D / 8); i += kSoftWarps * 32) {
-            const int t = i / (D / 8), c8 = i % (D / 8);
-            const int off = sw128_offset(gi * kGroup + t, c8);
-            *reinterpret_cast<uint4*>(&qs.k[t][8 * c8]) = *reinterpret_cast<const uint4*>(kt + off);
-            *reinterpret_cast<uint4*>(&qs.v[t][8 * c8]) = *reinterpret_cast<const uint4*>(vt + off);
-          }
-          sync();
-          uint8_t* rec = a.records + (seq * a.ngcap + g) * geo.bytes();
-          quant::quantize_tiles_to_record<D, BITS, kSoftWarps * 32>(
-              qs, reinterpret_cast<uint32_t*>(rec), r, sync);
-          sync();  // the tiles are refilled by the next group
-        } else {
-          // residual tokens t0 .. min(t0 + G, S) - 1 to ring slots t mod (R + G)
-          const int n = (t0 + kGroup < a.S ? t0 + kGroup : a.S) - t0;
-          for (int i = r; i < n * (D / 8); i += kSoftWarps * 32) {
-            const int t = t0 + i / (D / 8), c8 = i % (D / 8);
-            const int off = sw128_offset(t - qt * kTileN, c8);
-            const long dst = (seq * kRingSlots + t % kRingSlots) * D + 8 * c8;
-            *reinterpret_cast<uint4*>(a.ring_k + dst) = *reinterpret_cast<const uint4*>(kt + off);
-            *reinterpret_cast<uint4*>(a.ring_v + dst) = *reinterpret_cast<const uint4*>(vt + off);
+      const __nv_bfloat16* ks = a.k + seq * a.S * D;
+      const __nv_bfloat16* vs = a.v + seq * a.S * D;
+      auto sync = [] { named_sync(kQuantBarrier, kQuantThreadsPA); };
+      for (int u = 0; u < (partner == qt ? 1 : 2); ++u) {
+        const int tile = u == 0 ? qt : partner;
+        for (int gi = hi; gi < kTileN / kGroup; gi += nq) {
+          const int t0 = tile * kTileN + gi * kGroup;  // the group's first token
+          if (t0 >= a.S) break;
+          const int g = t0 / kGroup;
+          if (g < a.NG) {
+            quant::load_tile<D, kQuantThreadsPA>(qs.k, ks + (long)t0 * D, D, qtid);
+            quant::load_tile<D, kQuantThreadsPA>(qs.v, vs + (long)t0 * D, D, qtid);
+            sync();
+            uint8_t* rec = a.records + (seq * a.ngcap + g) * geo.bytes();
+            quant::quantize_tiles_to_record<D, BITS, kQuantThreadsPA>(
+                qs, reinterpret_cast<uint32_t*>(rec), qtid, sync);
+            sync();  // the tiles are refilled by the next group
+          } else {
+            // residual tokens t0 .. min(t0 + G, S) - 1 to ring slots t mod (R + G)
+            const int n = (t0 + kGroup < a.S ? t0 + kGroup : a.S) - t0;
+            for (int i = qtid; i < n * (D / 8); i += kQuantThreadsPA) {
+              const int t = t0 + i / (D / 8), c = i % (D / 8);
+              const long dst = (seq * kRingSlots + t % kRingSlots) * D;
+              reinterpret_cast<uint4*>(a.ring_k + dst)[c] =
+                  reinterpret_cast<const uint4*>(ks + (long)t * D)[c];
+              reinterpret_cast<uint4*>(a.ring_v + dst)[c] =
+                  reinterpret_cast<const uint4*>(vs + (long)t * D)[c];
+            }
           }
         }
       }
@@ -407,6 +469,8 @@ cudaError_t launch_pa_t(const PrefillAttnArgs& x, cudaStream_t stream) {
       !encode_bf16_map(&tv, x.v, (long)x.B * x.Hkv * x.S, D, kTileN))
     return cudaErrorInvalidValue;
   PAParams p{};
+  p.k = x.k;
+  p.v = x.v;
   p.out = x.out;
   p.status = x.status;
   p.B = x.B;

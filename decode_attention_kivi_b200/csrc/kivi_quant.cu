@@ -18,8 +18,8 @@ using quant::QuantSmem;
 
 constexpr int kQuantThreads = 128;
 
-template <int D>
-__device__ __forceinline__ void load_tile(__nv_bfloat16 (*dst)[D], const __nv_bfloat16* src,
+template <int D, int ROW>
+__device__ __forceinline__ void load_tile(__nv_bfloat16 (*dst)[ROW], const __nv_bfloat16* src,
                                           long ld) {
   quant::load_tile<D, kQuantThreads>(dst, src, ld, threadIdx.x);
 }

@@ -20,10 +20,14 @@
 namespace kivi {
 namespace quant {
 
+// The value rows are padded by 16 bytes: the per-token parameter loop, whose
+// threads read four channel blocks of eight tokens at once, then meets 4-way
+// bank conflicts instead of 16-way.
 template <int D>
 struct QuantSmem {
+  static constexpr int kVRow = D + 8;
   __nv_bfloat16 k[kGroup][D];
-  __nv_bfloat16 v[kGroup][D];
+  __nv_bfloat16 v[kGroup][kVRow];
   uint8_t kc[kGroup][D];
   uint8_t vc[kGroup][D];
 };
@@ -32,7 +36,8 @@ __device__ __forceinline__ unsigned short to_f16_bits(float x) {
   return __half_as_ushort(__float2half_rn(x));
 }
 
-// Codes of one group of values already reduced to (mn, scale).
+// Codes of one group of values already reduced to (mn, scale):
+// round-half-even(fl(fl(x - mn) / scale)), the quotient rounded to fp32 first.
 template <int BITS>
 __device__ __forceinline__ uint8_t quant_code(float x, float mn, float scale) {
   constexpr int kQmax = (1 << BITS) - 1;
@@ -41,11 +46,40 @@ __device__ __forceinline__ uint8_t quant_code(float x, float mn, float scale) {
   return (uint8_t)min(max(c, 0), kQmax);
 }
 
+// The same code with one multiply instead of the division, given inv =
+// fl(1 / scale).  With d = fl(x - mn) in [0, max - min], the quotient
+// Q = d / scale is at most 2^b - 1 (to within 2^-22), t = fl(d * inv) is within
+// 2^-19 of Q and fl(Q) within 2^-20 of Q.  So when t is more than 2^-12 away
+// from the nearest half-integer, fl(Q) lies on the same side of it and rounds
+// to the same integer as t; the rare rest (and a non-finite t, from an inverse
+// that overflows or is unusable) takes the division.
+template <int BITS>
+__device__ __forceinline__ uint8_t quant_code_inv(float x, float mn, float scale, float inv) {
+  constexpr int kQmax = (1 << BITS) - 1;
+  if (!(scale > 0.0f)) return 0;
+  const float d = __fsub_rn(x, mn);
+  float q = __fmul_rn(d, inv);
+  const float frac = q - floorf(q);  // NaN for a non-finite q: the test below fails
+  if (!(fabsf(frac - 0.5f) > 0x1p-12f)) q = __fdiv_rn(d, scale);
+  const int c = __float2int_rn(q);
+  return (uint8_t)min(max(c, 0), kQmax);
+}
+
+// fl(1 / scale) for quant_code_inv (unused when scale is 0); NaN, which sends
+// every code to the division, when the inverse would be subnormal and lose its
+// relative accuracy.
+__device__ __forceinline__ float quant_inverse(float scale) {
+  if (!(scale > 0.0f)) return 0.0f;
+  const float r = __fdiv_rn(1.0f, scale);
+  return r >= 0x1p-126f ? r : __int_as_float(0x7fffffff);
+}
+
 // Loads 32 token rows of D bf16 (row stride `ld` elements) into a smem tile,
 // with NT threads (tid in [0, NT)).
-template <int D, int NT>
-__device__ __forceinline__ void load_tile(__nv_bfloat16 (*dst)[D], const __nv_bfloat16* src,
+template <int D, int NT, int ROW>
+__device__ __forceinline__ void load_tile(__nv_bfloat16 (*dst)[ROW], const __nv_bfloat16* src,
                                           long ld, int tid) {
+  static_assert(ROW >= D && ROW * 2 % 16 == 0, "rows of whole 16-byte vectors");
   constexpr int kVecPerRow = D * 2 / 16;
   for (int i = tid; i < kGroup * kVecPerRow; i += NT) {
     const int t = i / kVecPerRow, c = i % kVecPerRow;
@@ -86,8 +120,10 @@ __device__ void quantize_tiles_to_record(QuantSmem<D>& sm, uint32_t* __restrict_
   for (int d = tid; d < D; d += NT) {
     float mn, scale;
     group_params<BITS>(&sm.k[0][d], kGroup, D, mn, scale);
+    const float inv = quant_inverse(scale);
 #pragma unroll 8
-    for (int t = 0; t < kGroup; ++t) sm.kc[t][d] = quant_code<BITS>(__bfloat162float(sm.k[t][d]), mn, scale);
+    for (int t = 0; t < kGroup; ++t)
+      sm.kc[t][d] = quant_code_inv<BITS>(__bfloat162float(sm.k[t][d]), mn, scale, inv);
     kscale[d] = to_f16_bits(scale);
     kmin[d] = to_f16_bits(mn);
   }
@@ -97,9 +133,11 @@ __device__ void quantize_tiles_to_record(QuantSmem<D>& sm, uint32_t* __restrict_
     const int t = p / kBlocks, j = p % kBlocks;
     float mn, scale;
     group_params<BITS>(&sm.v[t][32 * j], 32, 1, mn, scale);
+    const float inv = quant_inverse(scale);
 #pragma unroll 8
     for (int c = 0; c < 32; ++c)
-      sm.vc[t][32 * j + c] = quant_code<BITS>(__bfloat162float(sm.v[t][32 * j + c]), mn, scale);
+      sm.vc[t][32 * j + c] =
+          quant_code_inv<BITS>(__bfloat162float(sm.v[t][32 * j + c]), mn, scale, inv);
     vscale[v_meta_index(t, j)] = to_f16_bits(scale);
     vmin[v_meta_index(t, j)] = to_f16_bits(mn);
   }

@@ -12,28 +12,26 @@
 //   out[b][h][i] = sum_{j <= i} softmax_j(sm_scale * <q_i, k_j>) v_j.
 //
 // One CTA per (query tile of 128 positions, sequence, query head), the tiles
-// with the most key tiles first.  Twelve warps:
-//   warp 8 (producer)  2D tensor copies of Q once and of K and V tiles of 128
+// with the most key tiles first.  Eight warps:
+//   warp 4 (producer)  2D tensor copies of Q once and of K and V tiles of 128
 //                      keys into two-stage rings (128-byte swizzle), the
 //                      diagonal tile first, then towards key 0; a K stage is
 //                      refilled once its scores are computed, a V stage once
 //                      its product is;
-//   warp 9 (MMA)       one thread issues S_j = Q K_j^T (M = N = 128, K = D) into
+//   warp 5 (MMA)       one thread issues S_j = Q K_j^T (M = N = 128, K = D) into
 //                      one of two TMEM score buffers, and O += P_j V_j (M = 128,
 //                      N = D, K = 128) into the TMEM output, each followed by a
 //                      commit to an mbarrier;
-//   warps 0-7          half a query row per thread (warps w and w + 4 share the
-//                      TMEM lanes of rows 32 (w mod 4) + lane and take 64 keys
-//                      each): the row of S_j from TMEM, the causal mask on the
-//                      diagonal tile, the online softmax in base 2 (the halves
-//                      exchange their maxima once per tile) with the weights
-//                      computed while the tensor cores finish P_{j-1} V_{j-1},
-//                      then P_j as bf16 into shared memory in the operand layout
-//                      of the second MMA.  The output is rescaled in TMEM only
-//                      when a row maximum grew by more than 2^8 (up to then the
-//                      stale maximum is kept: the weights stay below 2^8 and
-//                      O / l is unchanged);
-//   warps 10-11        with the quantize on, in the CTAs of the longer half of
+//   warps 0-3          one query row per thread (its TMEM lane): the row of S_j
+//                      from TMEM, the causal mask on the diagonal tile, the
+//                      online softmax in base 2 with the weights computed while
+//                      the tensor cores finish P_{j-1} V_{j-1}, then P_j as bf16
+//                      into shared memory in the operand layout of the second
+//                      MMA.  The output is rescaled in TMEM only when a row
+//                      maximum grew by more than 2^8 (up to then the stale
+//                      maximum is kept: the weights stay below 2^8 and O / l is
+//                      unchanged);
+//   warps 6-7          with the quantize on, in the CTAs of the longer half of
 //                      the query tiles: this CTA's share of the groups of key
 //                      tiles qt and nqt - 1 - qt (query head j < 4 of a kv head
 //                      takes groups j, j + min(HPK, 4), ...): group records
@@ -62,13 +60,12 @@ namespace {
 
 constexpr int kTileM = 128;                   // query rows per CTA = TMEM lanes
 constexpr int kTileN = 128;                   // keys per tile
-constexpr int kSoftWarps = 8;                 // two per TMEM lane quarter: each row is split
-                                              // into two halves of 64 keys
-constexpr int kHalfN = kTileN / 2;
+constexpr int kSoftWarps = 4;
 constexpr int kProducerWarp = kSoftWarps;
 constexpr int kMmaWarp = kSoftWarps + 1;
 constexpr int kQuantWarp0 = kSoftWarps + 2;   // two warps that quantize the prompt
-constexpr int kQuantThreadsPA = 64;
+constexpr int kQuantThreadsPA = 64;           // (eight warps in all, two per SM sub-partition:
+                                              // up to 255 registers per thread)
 constexpr int kThreadsPA = (kSoftWarps + 2) * 32 + kQuantThreadsPA;
 constexpr int kSlabBytes = 128 * 128;         // 64 bf16 columns of 128 rows
 constexpr uint32_t kTmemCols = 512;
@@ -85,8 +82,7 @@ struct PACfg {
   static constexpr int kOffKV = kOffQ + kTileBytes;       // stage s: K at 2s, V at 2s + 1
   static constexpr int kOffP = kOffKV + 4 * kTileBytes;
   static constexpr int kOffQuant = kOffP + 2 * kSlabBytes; // P: 128 rows x 128 keys
-  static constexpr int kOffMax = kOffQuant + (int)sizeof(quant::QuantSmem<D>);  // [2][2][128] f32
-  static constexpr int kOffBars = kOffMax + 2 * 2 * kTileM * 4;
+  static constexpr int kOffBars = kOffQuant + (int)sizeof(quant::QuantSmem<D>);
   static constexpr int kUsed = kOffBars + 256;
   // more than half of the SM's shared memory: one CTA per SM, which holds all
   // 512 TMEM columns
@@ -139,8 +135,7 @@ prefill_attention_kernel(const __grid_constant__ CUtensorMap tq,
   uint64_t* p_full = q_full + 11;
   uint64_t* o_done = q_full + 12;
   uint64_t* drained = q_full + 13;
-  uint64_t* half_bar = q_full + 14;  // [4 lane quarters][2 tile parities]: row-max exchange
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(q_full + 22);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(q_full + 14);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -166,7 +161,6 @@ prefill_attention_kernel(const __grid_constant__ CUtensorMap tq,
     mbar_init(p_full, kSoftWarps * 32);
     mbar_init(o_done, 1);
     mbar_init(drained, 1);
-    for (int i = 0; i < 8; ++i) mbar_init(&half_bar[i], 64);
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -277,23 +271,17 @@ prefill_attention_kernel(const __grid_constant__ CUtensorMap tq,
       if (!mbar_wait_bounded(drained, 0)) fail();
     }
   } else if (warp < kSoftWarps) {
-    // Softmax warps: warps w and w + 4 share query rows 32 (w mod 4) + lane (their
-    // TMEM lanes); warp w takes keys [64 h, 64 h + 64) of each tile, h = w / 4.
-    // The two halves of a row exchange their maxima once per tile (through
-    // shared memory and an mbarrier, so a partner that stopped cannot hang it)
-    // and keep separate partial sums, added once at the end.
-    const int quarter = warp & 3, h = warp >> 2;
-    const int r = quarter * 32 + lane;
+    // Softmax warps: thread r owns query row r of the tile (TMEM lane r).
+    const int r = threadIdx.x;
     const int qpos = qt * kTileM + r;
-    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
     unsigned char* prow = smem + C::kOffP;
-    float* s_max = reinterpret_cast<float*>(smem + C::kOffMax);  // [parity][half][row]
     auto wait_warp = [&](uint64_t* bar, uint32_t parity) {
       const bool w = mbar_wait_bounded(bar, parity);
       return __all_sync(0xffffffffu, w && !*s_abort);
     };
     const float sl2 = a.scale_log2;
-    float m = -INFINITY, l = 0.f;  // running max (log2 units); this half's sum of weights
+    float m = -INFINITY, l = 0.f;  // running max (log2 units) and sum of the row's weights
     bool ok = true;
     for (int j = 0; j < nt; ++j) {
       const int st = j & 1;
@@ -302,38 +290,29 @@ prefill_attention_kernel(const __grid_constant__ CUtensorMap tq,
         break;
       }
       tc::fence_after();
-      float s[kHalfN];
-      tc::ld_x64(lane_base + C::kColS + st * kTileN + h * kHalfN, s);
+      float s[kTileN];
+      tc::ld_x128(lane_base + C::kColS + st * kTileN, s);
       if (j == 0) {  // the diagonal tile: keys after the query are masked
 #pragma unroll
-        for (int c = 0; c < kHalfN; ++c) s[c] = h * kHalfN + c <= r ? s[c] : -INFINITY;
+        for (int c = 0; c < kTileN; ++c) s[c] = c <= r ? s[c] : -INFINITY;
       }
       float mx8[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) mx8[i] = s[i];
 #pragma unroll
-      for (int c = 8; c < kHalfN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
-      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      // the other half's maximum (slot parity j: reused two tiles later, after
-      // the partner has passed the next exchange)
-      s_max[(st * 2 + h) * kTileM + r] = mx;
-      mbar_arrive(&half_bar[quarter * 2 + st]);
-      if (!wait_warp(&half_bar[quarter * 2 + st], (j >> 1) & 1)) {
-        ok = false;
-        break;
-      }
-      mx = fmaxf(mx, s_max[(st * 2 + (h ^ 1)) * kTileM + r]);
+      for (int c = 8; c < kTileN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       // scores scaled into log2 units inside the exponent's FMA (sl2 > 0 keeps the max)
       const float m_new = fmaxf(m, mx * sl2);
       const bool grow = m_new > m + kRescaleSlack;  // always at the first tile (m = -inf)
       const float m_use = grow ? m_new : m;
       const float alpha = fast_exp2(m - m_use);     // 1 when kept, 0 at the first tile
       // the weights of this tile while the tensor cores still work on the last one
-      uint32_t pk[kHalfN / 2];
+      uint32_t pk[kTileN / 2];
       float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < kHalfN; c += 2) {
+      for (int c = 0; c < kTileN; c += 2) {
         const float p0 = fast_exp2(fmaf(s[c], sl2, -m_use));
         const float p1 = fast_exp2(fmaf(s[c + 1], sl2, -m_use));
         sum4[(c >> 1) & 3] += p0 + p1;
@@ -348,7 +327,7 @@ prefill_attention_kernel(const __grid_constant__ CUtensorMap tq,
         tc::fence_after();
         if (__any_sync(0xffffffffu, grow)) {  // TMEM loads and stores are warp-wide
 #pragma unroll 1
-          for (int c0 = h * (D / 2); c0 < (h + 1) * (D / 2); c0 += 32) {
+          for (int c0 = 0; c0 < D; c0 += 32) {
             float o[32];
             tc::ld_x32(lane_base + C::kColO + c0, o);
 #pragma unroll
@@ -359,8 +338,8 @@ prefill_attention_kernel(const __grid_constant__ CUtensorMap tq,
         }
       }
 #pragma unroll
-      for (int c8 = 0; c8 < kHalfN / 8; ++c8)
-        *reinterpret_cast<uint4*>(prow + sw128_offset(r, h * (kHalfN / 8) + c8)) =
+      for (int c8 = 0; c8 < kTileN / 8; ++c8)
+        *reinterpret_cast<uint4*>(prow + sw128_offset(r, c8)) =
             make_uint4(pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]);
       l = l * alpha + ((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
       m = m_use;
@@ -370,20 +349,11 @@ prefill_attention_kernel(const __grid_constant__ CUtensorMap tq,
     }
     if (ok) ok = wait_warp(o_done, (nt - 1) & 1);
     if (ok) {
-      // the row's sum: this half's plus the other's (slot parity of tile nt,
-      // whose exchange never happens)
-      const int sp = nt & 1;
-      s_max[(sp * 2 + h) * kTileM + r] = l;
-      mbar_arrive(&half_bar[quarter * 2 + sp]);
-      ok = wait_warp(&half_bar[quarter * 2 + sp], (nt >> 1) & 1);
-      if (ok) l += s_max[(sp * 2 + (h ^ 1)) * kTileM + r];
-    }
-    if (ok) {
       tc::fence_after();
       const float inv = 1.f / l;
       float* orow = a.out + ((long)bh * a.S + qpos) * D;
 #pragma unroll 1
-      for (int c0 = h * (D / 2); c0 < (h + 1) * (D / 2); c0 += 32) {
+      for (int c0 = 0; c0 < D; c0 += 32) {
         float o[32];
         tc::ld_x32(lane_base + C::kColO + c0, o);
         if (qpos < a.S) {

@@ -522,3 +522,16 @@ def test_prefill_attention_equals_causal_sdpa(B, Hkv, Hq, S, D):
     np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
     # position 0 sees only token 0: its value row, exactly
     np.testing.assert_array_equal(out[:, :, 0], v.double().numpy().repeat(rep, 1)[:, :, 0])
+
+
+def test_prefill_attention_hand_worked():
+    """Two positions, D = 2, sm_scale = ln 3: position 1 scores (0, ln 3) against keys
+    (0, 0) and (1, 0), so its weights are 1/4 and 3/4 and its output is
+    v0/4 + 3 v1/4 = (1, 6) for v0 = (4, 0), v1 = (0, 8); position 0 sees only key 0 and
+    returns v0.  All inputs are exact in bf16."""
+    f = lambda a: _bits(torch.tensor(a, dtype=torch.float32).to(torch.bfloat16))  # noqa: E731
+    q = f([[[[5.0, -3.0], [1.0, 0.0]]]])
+    k = f([[[[0.0, 0.0], [1.0, 0.0]]]])
+    v = f([[[[4.0, 0.0], [0.0, 8.0]]]])
+    out = O.prefill_attention(q, k, v, sm_scale=math.log(3.0))
+    np.testing.assert_allclose(out[0, 0], [[4.0, 0.0], [1.0, 6.0]], rtol=0, atol=1e-12)
